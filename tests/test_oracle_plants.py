@@ -1,0 +1,28 @@
+"""Each deliberately wrong oracle build (a mistake planted in the C source
+behind ORACLE_PLANT=n, CPU only) must fail at least one pin; this shows the
+pins can see a dropped term, a wrong sign or index, or a transposed operand."""
+import pytest
+
+import pins
+
+PLANTS = {
+    1: "K smoothing dropped (km forced to 0)",
+    2: "Q/K scale and its inverse swapped",
+    3: "Q group of 64 rows instead of 32",
+    4: "log2(e) missing from the score scale",
+    5: "K channel index reversed in QK^T",
+    6: "old-max rescale of RO and d skipped",
+    7: "max not subtracted before exp2",
+    8: "V scale not applied in the epilogue",
+}
+
+
+@pytest.mark.parametrize("plant", sorted(PLANTS), ids=lambda n: f"plant{n}")
+def test_planted_mistake_is_caught(plant):
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(plant)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught planted mistake {plant}: {PLANTS[plant]}"

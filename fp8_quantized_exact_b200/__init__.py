@@ -1,0 +1,244 @@
+"""Python binding of the B200 quantized-attention C ABI (``include/sage_b200.h``).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+of ``libsage_b200.so``.  PyTorch supplies device memory and streams.  The
+functions keep the C names; tensors are passed where the C ABI takes device
+pointers, and a non-zero return code raises :class:`SageError`.
+
+There is no CPU fallback: if the shared library is missing or cannot be
+loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_build", "libsage_b200.so")
+
+SAGE_OK = 0
+SAGE_ERR_INVALID_ARG = 1
+SAGE_ERR_UNSUPPORTED = 2
+SAGE_ERR_WORKSPACE = 3
+SAGE_ERR_CUDA = 4
+SAGE_ERR_TIMEOUT = 5
+SAGE_ERR_DEVICE = 6
+
+SAGE_OP_QUANT_QK = 0
+SAGE_OP_QUANT_V = 1
+SAGE_OP_ATTN_FWD = 2
+SAGE_OP_ATTN_FROM_QUANT = 3
+SAGE_OP_DEBUG_QK = 4
+
+SAGE_MAINLOOP_DEFAULT = 0
+SAGE_MAINLOOP_TCGEN05 = 1
+SAGE_MAINLOOP_MMA_SYNC = 2
+
+SAGE_STATUS_BYTES = 256
+
+# every symbol the header declares (the CPU test checks the exports)
+EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_from_quant",
+           "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
+           "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32")
+
+
+class SageError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {sage_strerror(code)} (code {code})")
+
+
+class sage_view_bf16(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_n", ctypes.c_int64), ("stride_h", ctypes.c_int64)]
+
+
+class sage_fwd_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in
+                ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean", "v_fp8", "v_scale", "total")]
+
+
+_lib = None
+
+
+def lib():
+    """Load libsage_b200.so (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, L64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        V = sage_view_bf16
+        sig = {
+            "sage_workspace_bytes": [I, I, I, I, I, ctypes.POINTER(SZ)],
+            "sage_quant_qk": [V, V, I, I, I, I, P, P, P, P, P, P, SZ, P],
+            "sage_quant_v": [V, I, I, I, I, P, P, P, SZ, P],
+            "sage_attn_from_quant": [P, P, P, P, P, P, P, L64, L64, L64, I, I, I, I,
+                                     ctypes.c_float, P, SZ, P],
+            "sage_attn_fwd": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P, SZ, P],
+            "sage_fwd_workspace_layout": [I, I, I, I, ctypes.POINTER(sage_fwd_layout)],
+            "sage_read_device_status": [P, P],
+            "sage_strerror": [I],
+            "sage_set_mainloop": [I],
+            "sage_get_mainloop": [],
+            "sage_debug_qk_s32": [P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
+        }
+        for name, args in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = ctypes.c_char_p if name == "sage_strerror" else ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def sage_strerror(code: int) -> str:
+    try:
+        return lib().sage_strerror(int(code)).decode()
+    except Exception:  # the library itself is missing
+        return f"error {code}"
+
+
+def _check(rc: int, what: str):
+    if rc != SAGE_OK:
+        raise SageError(rc, what)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _view(t) -> sage_view_bf16:
+    import torch
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1 or not t.is_cuda:
+        raise ValueError("expected a CUDA bfloat16 [B, N, H, D] view with unit stride over D")
+    return sage_view_bf16(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+# ----------------------------------------------------------- C entry points
+def sage_workspace_bytes(op: int, B: int, N: int, H: int, D: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sage_workspace_bytes(op, B, N, H, D, ctypes.byref(n)), "sage_workspace_bytes")
+    return n.value
+
+
+def sage_fwd_workspace_layout(B: int, N: int, H: int, D: int) -> dict:
+    lay = sage_fwd_layout()
+    _check(lib().sage_fwd_workspace_layout(B, N, H, D, ctypes.byref(lay)), "sage_fwd_workspace_layout")
+    return {f: getattr(lay, f) for f, _ in sage_fwd_layout._fields_}
+
+
+def sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, workspace, stream=None):
+    B, N, H, D = q.shape
+    _check(lib().sage_quant_qk(_view(q), _view(k), B, N, H, D, _ptr(q_i8), _ptr(q_scale),
+                               _ptr(k_i8), _ptr(k_scale), _ptr(k_mean), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sage_quant_qk")
+
+
+def sage_quant_v(v, v_fp8, v_scale, workspace, stream=None):
+    B, N, H, D = v.shape
+    _check(lib().sage_quant_v(_view(v), B, N, H, D, _ptr(v_fp8), _ptr(v_scale), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sage_quant_v")
+
+
+def sage_attn_from_quant(q_i8, q_scale, k_i8, k_scale, v_fp8, v_scale, out, sm_scale, workspace,
+                         stream=None):
+    B, N, H, D = out.shape
+    _check(lib().sage_attn_from_quant(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale),
+                                      _ptr(v_fp8), _ptr(v_scale), _ptr(out), out.stride(0),
+                                      out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream)),
+           "sage_attn_from_quant")
+
+
+def sage_attn_fwd(q, k, v, out, sm_scale, workspace, stream=None):
+    B, N, H, D = q.shape
+    if out.stride(3) != 1 or tuple(out.shape) != (B, N, H, D):
+        raise ValueError("out must be [B, N, H, D] with unit stride over D")
+    _check(lib().sage_attn_fwd(_view(q), _view(k), _view(v), _ptr(out), out.stride(0),
+                               out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream)),
+           "sage_attn_fwd")
+
+
+def sage_read_device_status(workspace, stream=None) -> int:
+    return lib().sage_read_device_status(_ptr(workspace), _stream(stream))
+
+
+def sage_set_mainloop(which: int):
+    _check(lib().sage_set_mainloop(int(which)), "sage_set_mainloop")
+
+
+def sage_get_mainloop() -> int:
+    return lib().sage_get_mainloop()
+
+
+def sage_debug_qk_s32(q_i8, k_i8, B, N, H, D, b, h, q_tile, k_tile, s_out, workspace, stream=None):
+    _check(lib().sage_debug_qk_s32(_ptr(q_i8), _ptr(k_i8), B, N, H, D, b, h, q_tile, k_tile,
+                                   _ptr(s_out), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sage_debug_qk_s32")
+
+
+# ------------------------------------------------------- tensor conveniences
+def quant_shapes(B: int, N: int, H: int, D: int) -> dict:
+    """Shapes of the quantised buffers (layouts of include/sage_b200.h)."""
+    Nq = -(-N // 128) * 128
+    T64 = -(-N // 64)
+    Nk = T64 * 64
+    G32 = -(-N // 32)
+    return {"q_i8": (B, H, Nq, D), "q_scale": (B, H, G32), "k_i8": (B, H, Nk, D),
+            "k_scale": (B, H, T64), "k_mean": (B, H, D), "v_fp8": (B, H, D, Nk),
+            "v_scale": (B, H, D)}
+
+
+def workspace(op: int, B: int, N: int, H: int, D: int, device="cuda"):
+    """A workspace tensor for one call (uint8, 256-byte aligned by the allocator)."""
+    import torch
+    n = max(sage_workspace_bytes(op, B, N, H, D), SAGE_STATUS_BYTES)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def fwd_quant_views(ws, B: int, N: int, H: int, D: int) -> dict:
+    """Views of the quantised tensors that sage_attn_fwd leaves in its workspace."""
+    import torch
+    lay = sage_fwd_workspace_layout(B, N, H, D)
+    shp = quant_shapes(B, N, H, D)
+    dt = {"q_i8": torch.int8, "q_scale": torch.float32, "k_i8": torch.int8,
+          "k_scale": torch.float32, "k_mean": torch.float32, "v_fp8": torch.uint8,
+          "v_scale": torch.float32}
+    out = {}
+    for name, shape in shp.items():
+        n = 1
+        for s in shape:
+            n *= s
+        es = torch.empty((), dtype=dt[name]).element_size()
+        out[name] = ws[lay[name]:lay[name] + n * es].view(dt[name]).view(shape)
+    return out
+
+
+def attention(q, k, v, out=None, sm_scale: float = 0.0, ws=None, stream=None):
+    """Quantized attention of BF16 [B, N, H, D] CUDA views; returns BF16 [B, N, H, D]."""
+    import torch
+    B, N, H, D = q.shape
+    if out is None:
+        out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = workspace(SAGE_OP_ATTN_FWD, B, N, H, D, q.device)
+    sage_attn_fwd(q, k, v, out, sm_scale, ws, stream)
+    return out

@@ -1,0 +1,310 @@
+// C ABI of the library: argument checks, workspace carving, launches.
+// See include/sage_b200.h for the contract of every entry point.
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "sage_common.cuh"
+
+using namespace sage;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int g_mainloop = SAGE_MAINLOOP_DEFAULT;
+bool g_mainloop_env_read = false;
+
+struct Dims {
+  int B, N, H, D, Nq, Nk, G32, T64;
+};
+
+Dims make_dims(int B, int N, int H, int D) {
+  Dims d{B, N, H, D, 0, 0, 0, 0};
+  d.Nq = ceil_div(N, kQTile) * kQTile;
+  d.T64 = ceil_div(N, kKTile);
+  d.Nk = d.T64 * kKTile;
+  d.G32 = ceil_div(N, kQGroup);
+  return d;
+}
+
+int check_dims(int B, int N, int H, int D) {
+  if (B < 0 || N < 0 || H < 0 || D < 0) return SAGE_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  // keep every flat index inside int range assumptions of the kernels
+  if ((int64_t)B * H > (1 << 30) || N > (1 << 28)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+bool empty(int B, int N, int H) { return B == 0 || N == 0 || H == 0; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_view(const sage_view_bf16& v) {
+  if (!v.data) return SAGE_ERR_INVALID_ARG;
+  if (v.stride_b < 0 || v.stride_n < 0 || v.stride_h < 0) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(v.data) || (v.stride_b | v.stride_n | v.stride_h) & 7) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+int check_out(const void* out, int64_t sb, int64_t sn, int64_t sh) {
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  if (sb < 0 || sn < 0 || sh < 0) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(out) || (sb | sn | sh) & 7) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+// Byte offsets of every region of a workspace.
+struct Layout {
+  size_t status = 0;
+  size_t q8 = 0, q_scale = 0, k8 = 0, k_scale = 0, k_mean = 0, v8 = 0, v_scale = 0;
+  size_t k_part = 0, v_part = 0, v_amax = 0;
+  size_t total = 0;
+};
+
+Layout plan(int op, const Dims& d) {
+  Layout L;
+  size_t off = align_up(SAGE_STATUS_BYTES);
+  const size_t bh = (size_t)d.B * d.H;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  if (op == SAGE_OP_ATTN_FWD) {
+    L.q8 = take(bh * d.Nq * d.D);
+    L.q_scale = take(bh * d.G32 * sizeof(float));
+    L.k8 = take(bh * d.Nk * d.D);
+    L.k_scale = take(bh * d.T64 * sizeof(float));
+    L.k_mean = take(bh * d.D * sizeof(float));
+    L.v8 = take(bh * d.D * d.Nk);
+    L.v_scale = take(bh * d.D * sizeof(float));
+  }
+  if (op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
+  if (op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_V) {
+    L.v_part = take(bh * d.T64 * d.D * sizeof(float));
+    L.v_amax = take(bh * d.D * sizeof(float));
+  }
+  L.total = off;
+  return L;
+}
+
+int check_ws(void* ws, size_t bytes, size_t need) {
+  if (!ws) return SAGE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return SAGE_ERR_WORKSPACE;
+  if (bytes < need) return SAGE_ERR_WORKSPACE;
+  return SAGE_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int clear_status(void* ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, sizeof(DeviceStatus), s) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+float log2_scale(float sm_scale, int D) {
+  if (!(sm_scale > 0.0f)) sm_scale = (float)(1.0 / sqrt((double)D));
+  return (float)((double)sm_scale * 1.4426950408889634074);
+}
+
+int resolved_mainloop() {
+  if (!g_mainloop_env_read) {
+    g_mainloop_env_read = true;
+    const char* e = getenv("SAGE_MAINLOOP");
+    if (e && g_mainloop == SAGE_MAINLOOP_DEFAULT) {
+      if (!strcmp(e, "tcgen05")) g_mainloop = SAGE_MAINLOOP_TCGEN05;
+      else if (!strcmp(e, "mma_sync") || !strcmp(e, "mmasync")) g_mainloop = SAGE_MAINLOOP_MMA_SYNC;
+    }
+  }
+  if (g_mainloop == SAGE_MAINLOOP_DEFAULT) return tc_available() ? SAGE_MAINLOOP_TCGEN05 : SAGE_MAINLOOP_MMA_SYNC;
+  return g_mainloop;
+}
+
+AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const int8_t* k8,
+                       const float* ks, const uint8_t* v8, const float* vs, void* out,
+                       int64_t osb, int64_t osn, int64_t osh, float sm_scale, void* ws) {
+  AttnParams p;
+  p.q8 = q8; p.q_scale = qs; p.k8 = k8; p.k_scale = ks; p.v8 = v8; p.v_scale = vs;
+  p.out = static_cast<uint16_t*>(out);
+  p.os_b = osb; p.os_n = osn; p.os_h = osh;
+  p.B = d.B; p.N = d.N; p.H = d.H; p.D = d.D;
+  p.Nq = d.Nq; p.Nk = d.Nk; p.G32 = d.G32; p.T64 = d.T64;
+  p.sl2 = log2_scale(sm_scale, d.D);
+  p.status = static_cast<DeviceStatus*>(ws);
+  return p;
+}
+
+int run_mainloop(const AttnParams& p, cudaStream_t s) {
+  return resolved_mainloop() == SAGE_MAINLOOP_TCGEN05 ? launch_attn_tc(p, s) : launch_attn_mma(p, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int sage_workspace_bytes(int op, int B, int N, int H, int D, size_t* bytes) {
+  if (!bytes || op < SAGE_OP_QUANT_QK || op > SAGE_OP_DEBUG_QK) return SAGE_ERR_INVALID_ARG;
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  *bytes = plan(op, make_dims(B, N, H, D)).total;
+  return SAGE_OK;
+}
+
+int sage_fwd_workspace_layout(int B, int N, int H, int D, sage_fwd_layout* out) {
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  Layout L = plan(SAGE_OP_ATTN_FWD, make_dims(B, N, H, D));
+  out->q_i8 = L.q8; out->q_scale = L.q_scale; out->k_i8 = L.k8; out->k_scale = L.k_scale;
+  out->k_mean = L.k_mean; out->v_fp8 = L.v8; out->v_scale = L.v_scale; out->total = L.total;
+  return SAGE_OK;
+}
+
+int sage_quant_qk(sage_view_bf16 q, sage_view_bf16 k, int B, int N, int H, int D, int8_t* q_i8,
+                  float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(q)) || (rc = check_view(k))) return rc;
+  if (!q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(q_scale) || !aligned16(k_scale) ||
+      !aligned16(k_mean))
+    return SAGE_ERR_UNSUPPORTED;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_QUANT_QK, d);
+  if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  return launch_prepass_qk(q, k, B, N, H, D, q_i8, q_scale, k_i8, k_scale, k_mean,
+                           at<double>(workspace, L.k_part), s);
+}
+
+int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, float* v_scale,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(v))) return rc;
+  if (!v_fp8 || !v_scale) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(v_fp8) || !aligned16(v_scale)) return SAGE_ERR_UNSUPPORTED;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_QUANT_V, d);
+  if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  return launch_prepass_v(v, B, N, H, D, v_fp8, v_scale, at<float>(workspace, L.v_part),
+                          at<float>(workspace, L.v_amax), s);
+}
+
+int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                         const float* k_scale, const uint8_t* v_fp8, const float* v_scale,
+                         void* out, int64_t out_stride_b, int64_t out_stride_n,
+                         int64_t out_stride_h, int B, int N, int H, int D, float sm_scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v_fp8 || !v_scale) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v_fp8) || !aligned16(q_scale) ||
+      !aligned16(k_scale) || !aligned16(v_scale))
+    return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_out(out, out_stride_b, out_stride_n, out_stride_h))) return rc;
+  const Dims d = make_dims(B, N, H, D);
+  if ((rc = check_ws(workspace, workspace_bytes, plan(SAGE_OP_ATTN_FROM_QUANT, d).total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  return run_mainloop(make_params(d, q_i8, q_scale, k_i8, k_scale, v_fp8, v_scale, out,
+                                  out_stride_b, out_stride_n, out_stride_h, sm_scale, workspace),
+                      s);
+}
+
+int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* out,
+                  int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N,
+                  int H, int D, float sm_scale, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(q)) || (rc = check_view(k)) || (rc = check_view(v))) return rc;
+  if ((rc = check_out(out, out_stride_b, out_stride_n, out_stride_h))) return rc;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_ATTN_FWD, d);
+  if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  int8_t* q8 = at<int8_t>(workspace, L.q8);
+  float* qs = at<float>(workspace, L.q_scale);
+  int8_t* k8 = at<int8_t>(workspace, L.k8);
+  float* ks = at<float>(workspace, L.k_scale);
+  float* km = at<float>(workspace, L.k_mean);
+  uint8_t* v8 = at<uint8_t>(workspace, L.v8);
+  float* vs = at<float>(workspace, L.v_scale);
+  if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
+    return rc;
+  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_part),
+                             at<float>(workspace, L.v_amax), s)))
+    return rc;
+  return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
+                                  out_stride_h, sm_scale, workspace),
+                      s);
+}
+
+int sage_read_device_status(const void* workspace, void* stream) {
+  if (!workspace) return SAGE_ERR_INVALID_ARG;
+  DeviceStatus st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SAGE_ERR_CUDA;
+  return st.code;
+}
+
+const char* sage_strerror(int code) {
+  switch (code) {
+    case SAGE_OK: return "success";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or stride)";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported (head dim not 64/128, or a misaligned pointer or stride)";
+    case SAGE_ERR_WORKSPACE: return "workspace missing, not 256-byte aligned, or too small";
+    case SAGE_ERR_CUDA: return "a CUDA launch or runtime call failed";
+    case SAGE_ERR_TIMEOUT: return "a bounded device wait ran out (kernel abandoned its work)";
+    case SAGE_ERR_DEVICE: return "a kernel flagged an inconsistent device state";
+    default: return "unknown status code";
+  }
+}
+
+int sage_set_mainloop(int which) {
+  if (which < SAGE_MAINLOOP_DEFAULT || which > SAGE_MAINLOOP_MMA_SYNC) return SAGE_ERR_UNSUPPORTED;
+  g_mainloop = which;
+  g_mainloop_env_read = true;
+  return SAGE_OK;
+}
+
+int sage_get_mainloop(void) { return resolved_mainloop(); }
+
+int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int H, int D, int b,
+                      int h, int q_tile, int k_tile, int32_t* s_out, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  const Dims d = make_dims(B, N, H, D);
+  if (!q_i8 || !k_i8 || !s_out || empty(B, N, H)) return SAGE_ERR_INVALID_ARG;
+  if (b < 0 || b >= B || h < 0 || h >= H || q_tile < 0 || q_tile >= d.Nq / kQTile || k_tile < 0 ||
+      k_tile >= d.T64)
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(s_out)) return SAGE_ERR_UNSUPPORTED;
+  if ((rc = check_ws(workspace, workspace_bytes, plan(SAGE_OP_DEBUG_QK, d).total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  AttnParams p = make_params(d, q_i8, nullptr, k_i8, nullptr, nullptr, nullptr, nullptr, 0, 0, 0,
+                             0.0f, workspace);
+  return resolved_mainloop() == SAGE_MAINLOOP_TCGEN05
+             ? launch_debug_qk_tc(p, b, h, q_tile, k_tile, s_out, s)
+             : launch_debug_qk_mma(p, b, h, q_tile, k_tile, s_out, s);
+}
+
+}  // extern "C"

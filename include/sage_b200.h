@@ -1,0 +1,180 @@
+/*
+ * sage_b200.h — C ABI of the B200 (sm_100a) quantized attention library.
+ *
+ * The library computes SageAttention-2-style non-causal attention:
+ * INT8 Q K^T on tensor cores, an FP32 online softmax, FP8-E4M3 P V with an
+ * FP16 per-K32 instantaneous buffer added in order into an FP32 output
+ * accumulator, then 1/d normalisation, the V scale and a BF16 store.
+ *
+ * The operation is the one described in "Sage2 Blackwell Mainloop"
+ * (section "Existing Contract") and "State-Ownership Architecture
+ * Decision" (sections "Non-Negotiable Dataflow", the exact handoff record
+ * and "Interface And Future Ulysses Layout").  Where those pages leave a
+ * step open, this library takes the readings below:
+ *   - K mean: FP64 sum per (b,h,d), sequential in 64-token chunks, chunk
+ *     partials added in chunk order, km = float(sum / N).
+ *   - Q: 32 consecutive rows per scale; K (after subtracting km): 64 rows per
+ *     scale; both symmetric, scale = amax/127, byte = rint_even(x*(127/amax)).
+ *   - V: one scale per (b,h,d) over all tokens, scale = amax/448,
+ *     byte = E4M3 (OCP "FN", satfinite, round-to-nearest-even) of x*(448/amax).
+ *   - scores s = float(S) * fl32(fl32(q_scale*k_scale) * fl32(sm_scale*log2 e)),
+ *     base-2 exponentials, denominator summed from FP32 p before FP8.
+ *   - PV: keys 0-31 and 32-63 of each 64-key tile are two FP16 buffers, each
+ *     added into the FP32 accumulator in that order.
+ *   - out = bf16(fl32(fl32(RO * fl32(1/d)) * v_scale[d])).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device and
+ *     are owned by the caller.  The library allocates nothing, frees nothing
+ *     and does not synchronise (except sage_read_device_status).  Work is
+ *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Shapes: B (batch), N (tokens), H (heads), D (head dim, 64 or 128).
+ *     B, N or H equal to 0 is an empty problem: SAGE_OK, nothing launched.
+ *   - BF16 views carry element strides (b, n, h); d has unit stride.  The
+ *     base address and every stride must be 16-byte aligned (strides a
+ *     multiple of 8 elements); three views may alias one fused projection
+ *     buffer.  No input copy or transpose is made.
+ *   - Return codes are synchronous argument / launch checks.  Faults found
+ *     on the device (a bounded wait that ran out) are written to the status
+ *     block at the start of the workspace; read them with
+ *     sage_read_device_status.
+ *   - Outputs are fully overwritten, padding included.
+ *
+ * Quantised buffer layouts (all 16-byte aligned, written by the prepasses):
+ *   Nq = ceil(N/128)*128, Nk = ceil(N/64)*64, G32 = ceil(N/32), T64 = Nk/64
+ *   q_i8    int8   [B][H][Nq][D]   rows >= N are zero
+ *   q_scale float  [B][H][G32]
+ *   k_i8    int8   [B][H][Nk][D]   smoothed (K - k_mean); rows >= N zero
+ *   k_scale float  [B][H][T64]
+ *   k_mean  float  [B][H][D]
+ *   v_fp8   uint8  [B][H][D][Nk]   E4M3, transposed (tokens contiguous);
+ *                                  tokens >= N zero
+ *   v_scale float  [B][H][D]
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum sage_status_code {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad stride */
+  SAGE_ERR_UNSUPPORTED = 2,  /* D not in {64, 128}; misaligned base or stride */
+  SAGE_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
+  SAGE_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+  SAGE_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out */
+  SAGE_ERR_DEVICE = 6        /* device status: a kernel flagged bad state */
+};
+
+/* Which call a workspace is sized for. */
+enum sage_op {
+  SAGE_OP_QUANT_QK = 0,
+  SAGE_OP_QUANT_V = 1,
+  SAGE_OP_ATTN_FWD = 2,
+  SAGE_OP_ATTN_FROM_QUANT = 3,
+  SAGE_OP_DEBUG_QK = 4
+};
+
+/* Mainloop implementations (same numerics, chosen by measurement). */
+enum sage_mainloop {
+  SAGE_MAINLOOP_DEFAULT = 0, /* the fastest validated variant */
+  SAGE_MAINLOOP_TCGEN05 = 1, /* tcgen05 MMAs with TMEM accumulators, TMA */
+  SAGE_MAINLOOP_MMA_SYNC = 2 /* warp-level mma.sync */
+};
+
+/* Bytes at the start of every workspace that hold the device status word. */
+#define SAGE_STATUS_BYTES 256
+
+/* A strided BF16 [B, N, H, D] view (element strides; unit stride over d). */
+typedef struct sage_view_bf16 {
+  const void* data;
+  int64_t stride_b, stride_n, stride_h;
+} sage_view_bf16;
+
+/* Workspace size for one call `op` on a (B, N, H, D) problem.
+ * Returns SAGE_OK and writes *bytes, or SAGE_ERR_INVALID_ARG. */
+SAGE_API int sage_workspace_bytes(int op, int B, int N, int H, int D, size_t* bytes);
+
+/* Prepasses for Q and K: K channel mean (FP64, reading above), K smoothing
+ * and per-64-row INT8 K, per-32-row INT8 Q.  Defined by "Sage2 Blackwell
+ * Mainloop", sections "Decision" (K mean/smoothing, Q quantization, K
+ * subtract-mean quantization) and "Existing Contract".
+ * Outputs use the layouts above.  Workspace: sage_workspace_bytes(
+ * SAGE_OP_QUANT_QK, ...) bytes, 256-byte aligned. */
+SAGE_API int sage_quant_qk(sage_view_bf16 q, sage_view_bf16 k, int B, int N, int H, int D,
+                  int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Prepass for V: per-channel amax over all tokens, scale, E4M3 bytes stored
+ * transposed.  Defined by "Sage2 Blackwell Mainloop", section "Decision"
+ * (V transpose/pad/permute, V scale/FP8 quantization) and section
+ * "Completed P1 And P2" (one owned direct-NHD V producer).
+ * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_V, ...). */
+SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, float* v_scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Fused mainloop on quantised inputs: every 64-key tile in increasing order,
+ * INT8 QK^T, score scaling, online softmax, E4M3 P, two K32 FP16 PV buffers
+ * added into FP32, then 1/d, V scale and the BF16 store to `out`
+ * ([B, N, H, D] with element strides out_stride_*; unit stride over d).
+ * Defined by "State-Ownership Architecture Decision", section
+ * "Non-Negotiable Dataflow" and the exact handoff record.
+ * sm_scale <= 0 selects 1/sqrt(D).
+ * Workspace: sage_workspace_bytes(SAGE_OP_ATTN_FROM_QUANT, ...). */
+SAGE_API int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
+                         const float* k_scale, const uint8_t* v_fp8, const float* v_scale,
+                         void* out, int64_t out_stride_b, int64_t out_stride_n,
+                         int64_t out_stride_h, int B, int N, int H, int D, float sm_scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole path: both prepasses (quantised tensors kept in the workspace)
+ * then the fused mainloop.  Workspace: sage_workspace_bytes(
+ * SAGE_OP_ATTN_FWD, ...) bytes, 256-byte aligned. */
+SAGE_API int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* out,
+                  int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N,
+                  int H, int D, float sm_scale, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Where the quantised tensors of sage_attn_fwd live inside its workspace
+ * (byte offsets from the workspace base, layouts above). */
+typedef struct sage_fwd_layout {
+  size_t q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale, total;
+} sage_fwd_layout;
+SAGE_API int sage_fwd_workspace_layout(int B, int N, int H, int D, sage_fwd_layout* layout);
+
+/* Synchronises `stream`, then returns the device status word stored at the
+ * start of `workspace` (SAGE_OK, SAGE_ERR_TIMEOUT, SAGE_ERR_DEVICE) or
+ * SAGE_ERR_CUDA if the copy fails.  The word is cleared by each call that
+ * uses the workspace. */
+SAGE_API int sage_read_device_status(const void* workspace, void* stream);
+
+/* Static English text for a return code. */
+SAGE_API const char* sage_strerror(int code);
+
+/* Select the mainloop used by sage_attn_fwd / sage_attn_from_quant for the
+ * calling process.  Returns SAGE_ERR_UNSUPPORTED for an unknown value. */
+SAGE_API int sage_set_mainloop(int which);
+SAGE_API int sage_get_mainloop(void);
+
+/* Test export: the int32 Q K^T tile that the selected mainloop computes for
+ * query tile q_tile (128 rows) and key tile k_tile (64 keys) of head (b, h),
+ * written to s_out[128][64] (device, row-major, natural key order). */
+SAGE_API int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int H, int D, int b,
+                      int h, int q_tile, int k_tile, int32_t* s_out, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_B200_H */

@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI that need no GPU: the library builds and
+loads, exports every function include/sage_b200.h declares, sizes
+workspaces, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import fp8_quantized_exact_b200 as sage
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp8_quantized_exact_b200 import build
+    build.build()
+    return sage.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"SAGE_API\s+[\w\s\*]+?\b(sage_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == set(sage.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_workspace_sizes(lib):
+    # long-context fused config: B1 N37810 H56 D128
+    n = sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD, 1, 37810, 56, 128)
+    bh, Nq, Nk, T = 56, 37888, 37824, 591
+    quant = bh * (Nq * 128 + Nk * 128 + 128 * Nk)
+    assert quant + bh * T * 128 * 12 < n < quant + bh * T * 128 * 12 + (2 << 20)
+    assert sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FROM_QUANT, 1, 37810, 56, 128) < 4096
+    assert sage.sage_workspace_bytes(sage.SAGE_OP_QUANT_QK, 2, 1000, 8, 64) >= 2 * 8 * 16 * 64 * 8
+    lay = sage.sage_fwd_workspace_layout(1, 1000, 8, 128)
+    offs = [lay[k] for k in ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean", "v_fp8", "v_scale")]
+    assert offs == sorted(offs) and all(o % 1024 == 0 for o in offs) and offs[0] >= 256
+    assert lay["total"] == sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD, 1, 1000, 8, 128)
+
+
+def test_argument_errors_need_no_device(lib):
+    assert sage.sage_strerror(0) == "success"
+    n = ctypes.c_size_t()
+    assert lib.sage_workspace_bytes(2, 1, 100, 2, 96, ctypes.byref(n)) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_workspace_bytes(2, -1, 100, 2, 64, ctypes.byref(n)) == sage.SAGE_ERR_INVALID_ARG
+    assert lib.sage_workspace_bytes(9, 1, 100, 2, 64, ctypes.byref(n)) == sage.SAGE_ERR_INVALID_ARG
+    null = sage.sage_view_bf16(None, 0, 0, 0)
+    good = sage.sage_view_bf16(4096, 256 * 2 * 128, 2 * 128, 128)
+    odd = sage.sage_view_bf16(4096 + 2, 256 * 2 * 128, 2 * 128, 128)
+    badstride = sage.sage_view_bf16(4096, 256 * 2 * 128, 2 * 128 + 4, 128)
+    fwd = lib.sage_attn_fwd
+    # empty problems succeed and launch nothing
+    assert fwd(null, null, null, None, 0, 0, 0, 0, 10, 2, 128, 0.0, None, 0, None) == sage.SAGE_OK
+    assert fwd(null, null, null, None, 0, 0, 0, 1, 0, 2, 128, 0.0, None, 0, None) == sage.SAGE_OK
+    assert fwd(null, good, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096, 1 << 20, None) == sage.SAGE_ERR_INVALID_ARG
+    assert fwd(good, good, good, 4096, 0, 0, 0, 1, 10, 2, 100, 0.0, 4096, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert fwd(odd, good, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert fwd(good, badstride, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096, 1 << 20, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert fwd(good, good, good, None, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096, 1 << 20, None) == sage.SAGE_ERR_INVALID_ARG
+    # workspace missing, misaligned, too small
+    assert fwd(good, good, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, None, 1 << 20, None) == sage.SAGE_ERR_WORKSPACE
+    assert fwd(good, good, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096 + 16, 1 << 20, None) == sage.SAGE_ERR_WORKSPACE
+    assert fwd(good, good, good, 4096, 0, 0, 0, 1, 10, 2, 128, 0.0, 4096, 100, None) == sage.SAGE_ERR_WORKSPACE
+    fq = lib.sage_attn_from_quant
+    assert fq(None, 4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
+    assert fq(4096, 4096, 4096 + 8, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_set_mainloop(7) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_debug_qk_s32(4096, 4096, 1, 100, 2, 64, 0, 2, 0, 0, 4096, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sage, "_lib", None)
+    monkeypatch.setattr(sage, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        sage.lib()

@@ -40,7 +40,9 @@ SAGE_STATUS_BYTES = 256
 # every symbol the header declares (the CPU test checks the exports)
 EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
-           "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32")
+           "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
+           "sage_attn_fwd_noalloc")
+SAGE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class SageError(RuntimeError):
@@ -85,6 +87,7 @@ def lib():
             "sage_set_mainloop": [I],
             "sage_get_mainloop": [],
             "sage_debug_qk_s32": [P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
+            "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -174,6 +177,19 @@ def sage_attn_fwd(q, k, v, out, sm_scale, workspace, stream=None):
                                _ptr(workspace), workspace.numel() * workspace.element_size(),
                                _stream(stream)),
            "sage_attn_fwd")
+
+
+def sage_attn_fwd_noalloc(q, k, v, out, sm_scale, stream=None):
+    """sage_attn_fwd without a workspace, for callers that cannot allocate
+    device memory: the scratch is a fixed array inside the library (see the
+    header for the size limit and the rule that overlapping calls race)."""
+    B, N, H, D = q.shape
+    if out.stride(3) != 1 or tuple(out.shape) != (B, N, H, D):
+        raise ValueError("out must be [B, N, H, D] with unit stride over D")
+    _check(lib().sage_attn_fwd_noalloc(_view(q), _view(k), _view(v), _ptr(out), out.stride(0),
+                                       out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
+                                       _stream(stream)),
+           "sage_attn_fwd_noalloc")
 
 
 def sage_read_device_status(workspace, stream=None) -> int:

@@ -167,6 +167,33 @@ SAGE_API const char* sage_strerror(int code);
 SAGE_API int sage_set_mainloop(int which);
 SAGE_API int sage_get_mainloop(void);
 
+/* Size of the fixed device array behind sage_attn_fwd_noalloc (64 MiB). */
+#define SAGE_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* sage_attn_fwd for callers that cannot allocate device memory (no
+ * counterpart in the pages: it is a packaging of the same path).  Some
+ * callers have no way to obtain a workspace: they run where cudaMalloc is
+ * not allowed, or inside a framework that owns all device memory, or are
+ * handed tensors but no allocator.  This entry point takes the same
+ * arguments as sage_attn_fwd minus the workspace and uses instead one fixed
+ * array of SAGE_NOALLOC_SCRATCH_BYTES compiled into the library, which every
+ * GPU that loads the library keeps until the process exits.  It allocates
+ * and frees nothing.
+ *   - Problems whose sage_workspace_bytes(SAGE_OP_ATTN_FWD, ...) exceeds
+ *     SAGE_NOALLOC_SCRATCH_BYTES are rejected with SAGE_ERR_WORKSPACE before
+ *     anything is launched (B*H*N*D of roughly 20 million or fewer fits).
+ *   - The first call on a device looks up the array's device address on
+ *     that device (the device must be current); make that first call before
+ *     any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     each call rewrites every byte it reads.  Calls whose work can overlap
+ *     on the GPU (different streams, or different host threads on one
+ *     device) race on the array and must be serialised by the caller. */
+SAGE_API int sage_attn_fwd_noalloc(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v,
+                                   void* out, int64_t out_stride_b, int64_t out_stride_n,
+                                   int64_t out_stride_h, int B, int N, int H, int D,
+                                   float sm_scale, void* stream);
+
 /* Test export: the int32 Q K^T tile that the selected mainloop computes for
  * query tile q_tile (128 rows) and key tile k_tile (64 keys) of head (b, h),
  * written to s_out[128][64] (device, row-major, natural key order). */

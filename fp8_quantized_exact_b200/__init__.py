@@ -41,7 +41,7 @@ SAGE_STATUS_BYTES = 256
 EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
            "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
-           "sage_attn_fwd_noalloc")
+           "sage_attn_fwd_noalloc", "sage_debug_set_stall")
 SAGE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -88,6 +88,7 @@ def lib():
             "sage_get_mainloop": [],
             "sage_debug_qk_s32": [P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
             "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
+            "sage_debug_set_stall": [I, ctypes.c_longlong],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -189,7 +190,7 @@ def sage_attn_fwd_noalloc(q, k, v, out, sm_scale, stream=None):
     _check(lib().sage_attn_fwd_noalloc(_view(q), _view(k), _view(v), _ptr(out), out.stride(0),
                                        out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
                                        _stream(stream)),
-           "sage_attn_fwd_noalloc")
+           "sage_attn_fwd_noalloc", "sage_debug_set_stall")
 
 
 def sage_read_device_status(workspace, stream=None) -> int:
@@ -202,6 +203,10 @@ def sage_set_mainloop(which: int):
 
 def sage_get_mainloop() -> int:
     return lib().sage_get_mainloop()
+
+
+def sage_debug_set_stall(k_tile: int, wait_limit_cycles: int = 0):
+    _check(lib().sage_debug_set_stall(int(k_tile), int(wait_limit_cycles)), "sage_debug_set_stall")
 
 
 def sage_debug_qk_s32(q_i8, k_i8, B, N, H, D, b, h, q_tile, k_tile, s_out, workspace, stream=None):

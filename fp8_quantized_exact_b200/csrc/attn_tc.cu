@@ -2,22 +2,27 @@
 // TMA), sm_100a.
 //
 // One CTA = one 128-row query tile of one (b, h); ten warps with fixed roles
-// (the ownership split of the pages' VEA-B design, built with TMEM instead of
-// register-resident accumulators):
+// (the ownership split of the pages' VEA-B design, built on TMEM):
 //   warps 0-3  QK/softmax owners: thread i owns query row i (TMEM lane i), its
 //              running max m and denominator d.  Per tile they read the int32
 //              scores from TMEM, scale them, update m, d and the rescale
 //              factor r, and write the E4M3 probabilities back to TMEM.
-//   warps 4-7  PV/output owners: thread i owns the FP32 output row RO of row
-//              i in registers; per tile it applies r, then adds each of the
-//              two FP16 K32 PV buffers (read from TMEM) in order; at the end
-//              it applies 1/d and the V scale and stores BF16.
+//   warps 4-7  output owners: per tile they apply r to the FP32 output row RO
+//              (kept in TMEM) when the max moved, and repack each FP16 K32 PV
+//              buffer in place into the packed FP16 operand layout; at the end
+//              they apply 1/d and the V scale and store BF16.
 //   warp 8     TMA producer: the Q tile once, then K and V^T tiles of 64 keys
 //              into a ring of shared-memory stages.
-//   warp 9     MMA issuer (one thread): per tile one INT8 QK^T MMA chain into
-//              a TMEM score buffer, and per K32 slice one E4M3 MMA with the
-//              probabilities as the TMEM A operand into an FP16 accumulator
-//              that starts at zero.
+//   warp 9     MMA issuer (one thread), per tile: one INT8 QK^T MMA chain into
+//              a TMEM score buffer (two tiles ahead of PV); per K32 slice one
+//              E4M3 MMA, with the probabilities as the TMEM A operand, into an
+//              FP16 accumulator that starts at zero (the instantaneous buffer);
+//              then, per slice, FP16 MMAs of that buffer against a 16x16
+//              identity held in shared memory accumulate it into the FP32 RO.
+//              With one non-zero product per output, each of those adds the
+//              FP16 value exactly to RO with one FP32 rounding in the tensor
+//              core: the ordered "RO += float(tmp)" per slice, done on the
+//              tensor pipe instead of two ALU instructions per element.
 // Handoffs are block-scope mbarriers; tcgen05.commit signals MMA completion.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in
 // the status word, raises a CTA-wide abort flag, and every role then leaves
@@ -42,22 +47,24 @@ constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns
-constexpr uint32_t kColO = 256;    // two FP16 PV buffers of D columns
-constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
+constexpr uint32_t kColRO = 128;   // FP32 output accumulator, D columns
+constexpr uint32_t kColO = 256;    // two FP16 PV buffers of 128 columns (one per K32 slice)
 
 template <int D>
 struct TcSmem {
   alignas(1024) uint8_t q[kQTile * D];
   alignas(1024) uint8_t k[kStages][kKTile * D];
   alignas(1024) uint8_t v[kStages][D * kKTile];
+  alignas(1024) uint16_t ident[16 * 16];  // FP16 16x16 identity, K-major, no swizzle
   float r_ring[2][kQTile];
   float rcp[kQTile];
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_full[2], o_free[2];
+  uint64_t o_full[2], o_packed[2], o_free[2];
+  uint64_t ro_ready, id_done;
   uint64_t done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -87,13 +94,14 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 // Bounded wait.  Returns false if the CTA is aborting or the wait ran out
 // (then the status word and the abort flag are set).
 __device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          DeviceStatus* st, int where, bool honour_abort = true) {
+                                             DeviceStatus* st, int where, long long limit,
+                                             bool honour_abort = true) {
   const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try(b, parity)) return true;
     if ((i & 31u) == 31u) {
       if (honour_abort && *abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) break;
+      if (clock64() - t0 > limit) break;
     }
   }
   *abort_flag = 1;
@@ -202,6 +210,61 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
+#define SAGE_R32(r) "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
+    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),   \
+    "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),              \
+    "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),              \
+    "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define SAGE_W32(r) "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), \
+    "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),            \
+    "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),          \
+    "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+#define SAGE_REGS32 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}"
+#define SAGE_REGS32_1 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32}"
+
+// 32 lanes x 32 columns of 32 bits -> 32 registers.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " SAGE_REGS32 ", [%32];" : SAGE_R32(r) : "r"(taddr));
+}
+// 32 registers -> 32 lanes x 32 columns.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], " SAGE_REGS32_1 ";" ::"r"(taddr), SAGE_W32(r)
+               : "memory");
+}
+// 64 columns of FP16 values (one per 32-bit column) -> 32 registers, two per
+// register (column 2j in the low half).
+__device__ __forceinline__ void tmem_ld32_pack16(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.pack::16b.b32 " SAGE_REGS32 ", [%32];"
+               : SAGE_R32(r)
+               : "r"(taddr));
+}
+
+// FP16 x FP16 -> FP32 MMA with A in TMEM (M = 128).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;}" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Descriptor of a K-major tile without swizzle: 8-row x 16-byte core
+// matrices, `lbo` bytes apart along K and `sbo` bytes apart along M/N.
+__device__ __forceinline__ uint64_t smem_desc_noswz(const void* tile, uint32_t lbo, uint32_t sbo) {
+  const uint32_t a = smem_u32(tile);
+  uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;  // layout type 0: no swizzle
+}
+
+// Identity MMA: F16 x F16 -> F32, M = 128, N = 16.
+__host__ __device__ constexpr uint32_t idesc_id() {
+  return (1u << 4) | ((uint32_t)(16 >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -238,6 +301,61 @@ __device__ __forceinline__ TcSmem<D>& tc_smem() {
 }
 
 // ------------------------------------------------------------------ kernel
+// Softmax of one tile for one row (TAIL: keys >= nvalid are masked).
+// In: S[64] int32 scores.  Out: P[16] packed E4M3 probabilities; updates
+// m and d, returns r (the factor applied to the older RO and d).
+template <bool TAIL>
+__device__ __forceinline__ float softmax_tile(const uint32_t (&S)[64], float cs, int nvalid, float& m,
+                                              float& d, uint32_t (&P)[16]) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
+  float fb[64];
+#pragma unroll
+  for (int j = 0; j < 64; ++j) {
+    fb[j] = __int_as_float((int32_t)S[j] + 0x4B400000);
+    if (TAIL && j >= nvalid) fb[j] = -INFINITY;
+  }
+  // tile max over the exact float images of the scores (3-input max)
+  float mx[22];
+#pragma unroll
+  for (int j = 0; j < 21; ++j) mx[j] = fmaxf(fmaxf(fb[3 * j], fb[3 * j + 1]), fb[3 * j + 2]);
+  mx[21] = fb[63];
+#pragma unroll
+  for (int j = 0; j < 7; ++j) mx[j] = fmaxf(fmaxf(mx[3 * j], mx[3 * j + 1]), mx[3 * j + 2]);
+  const float fmx = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[21])));
+  // max of fl32(S*c) = fl32(max(S)*c) since rounding is monotone and c >= 0
+  const float tmax = __fmul_rn(__fsub_rn(fmx, kMagic), cs);
+  const float m_new = fmaxf(m, tmax);
+  const float r = (m_new == m) ? 1.0f : ex2(__fsub_rn(m, m_new));
+  m = m_new;
+  // exponent argument s - m_new as one FMA on the float image:
+  // fb*c - (magic*c + m_new), with magic*c + m_new rounded once
+  const float kofs = __fmaf_rn(kMagic, cs, m_new);
+  float rs[2] = {0.0f, 0.0f};
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * q + e;
+      pv[e] = ex2(__fmaf_rn(fb[j], cs, -kofs));
+      if (TAIL && j >= nvalid) pv[e] = 0.0f;
+    }
+    // two independent packed FP32 sums (pairs of lanes of an f32x2 add)
+    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
+        " mov.b64 {%0, %1}, a;}"
+        : "+f"(rs[0]), "+f"(rs[1])
+        : "f"(pv[0]), "f"(pv[1]));
+    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
+        " mov.b64 {%0, %1}, a;}"
+        : "+f"(rs[0]), "+f"(rs[1])
+        : "f"(pv[2]), "f"(pv[3]));
+    P[q] = (uint32_t)e4m3x2(pv[0], pv[1]) | ((uint32_t)e4m3x2(pv[2], pv[3]) << 16);
+  }
+  d = __fadd_rn(__fmul_rn(d, r), __fadd_rn(rs[0], rs[1]));
+  return r;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -261,12 +379,25 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.p_full[i], kQTile);
       mbar_init(&sm.r_free[i], kQTile);
       mbar_init(&sm.o_full[i], 1);
-      mbar_init(&sm.o_free[i], kQTile);
+      mbar_init(&sm.o_packed[i], kQTile);
+      mbar_init(&sm.o_free[i], 1);
     }
+    mbar_init(&sm.ro_ready, kQTile);
+    mbar_init(&sm.id_done, 1);
     mbar_init(&sm.done, kQTile);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kLoadWarp) {
+    // FP16 identity in the no-swizzle K-major layout: element (n, k) at
+    // (n/8)*256 + (k/8)*128 + (n%8)*16 + (k%8)*2 bytes
+    for (int e = lane; e < 256; e += 32) {
+      const int n = e >> 4, k = e & 15;
+      sm.ident[((n >> 3) * 256 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) / 2] =
+          (n == k) ? (uint16_t)0x3C00u : (uint16_t)0u;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
@@ -276,12 +407,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
   if (warp < 4) {
     // ------------------------------------------------ QK / softmax owners
-    const int i = threadIdx.x;                      // row within the tile = TMEM lane
+    const int i = threadIdx.x;  // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
     const int row = qt * kQTile + i;
     const int grp = row / kQGroup;
     const float qs = grp < p.G32 ? p.q_scale[(size_t)bh * p.G32 + grp] : 0.0f;
     const float* ksc = p.k_scale + (size_t)bh * T;
+    const int ntail = p.N - (T - 1) * kKTile;  // valid keys of the last tile
     float m = -INFINITY, d = 0.0f;
     float ks_next = ksc[0];
     for (int t = 0; t < T; ++t) {
@@ -289,49 +421,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const uint32_t ph = (t >> 1) & 1;
       const float ks = ks_next;
       if (t + 1 < T) ks_next = ksc[t + 1];
-      if (!wait_bounded(&sm.s_full[bi], ph, abort_flag, p.status, 1)) break;
+      if (!wait_bounded(&sm.s_full[bi], ph, abort_flag, p.status, 1, p.wait_limit)) break;
       tc_fence_after();
       uint32_t S[64];
       tmem_ld64(lane_addr + kColS + 64 * bi, S);
       tmem_wait_ld();
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
-      const int nvalid = min(kKTile, p.N - t * kKTile);
-      int imax = INT_MIN;
-      if (nvalid == kKTile) {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) imax = max(imax, (int)S[j]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 64; ++j)
-          if (j < nvalid) imax = max(imax, (int)S[j]);
-      }
-      // the max of fl32(S*c) is fl32(max(S)*c): rounding is monotone, c >= 0
-      const float tmax = __fmul_rn(__int2float_rn(imax), cs);
-      const float m_new = fmaxf(m, tmax);
-      const float r = (m_new == m) ? 1.0f : ex2(__fsub_rn(m, m_new));
-      d = __fmul_rn(d, r);
-      float rs0 = 0.0f, rs1 = 0.0f;
       uint32_t P[16];
-#pragma unroll
-      for (int qd = 0; qd < 16; ++qd) {
-        float pv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int j = 4 * qd + e;
-          const float s = __fmul_rn(i2f_small((int32_t)S[j]), cs);
-          float pj = ex2(__fsub_rn(s, m_new));
-          if (nvalid != kKTile && j >= nvalid) pj = 0.0f;
-          pv[e] = pj;
-        }
-        rs0 = __fadd_rn(rs0, __fadd_rn(pv[0], pv[1]));
-        rs1 = __fadd_rn(rs1, __fadd_rn(pv[2], pv[3]));
-        P[qd] = (uint32_t)e4m3x2(pv[0], pv[1]) | ((uint32_t)e4m3x2(pv[2], pv[3]) << 16);
-      }
-      d = __fadd_rn(d, __fadd_rn(rs0, rs1));
-      m = m_new;
+      float r;
+      if (t + 1 < T || ntail == kKTile) r = softmax_tile<false>(S, cs, kKTile, m, d, P);
+      else r = softmax_tile<true>(S, cs, ntail, m, d, P);
       tmem_st16(lane_addr + kColS + 64 * bi, P);  // E4M3 P over the first 16 score columns
       tmem_wait_st();
-      if (!wait_bounded(&sm.r_free[bi], ph ^ 1u, abort_flag, p.status, 2)) break;
+      if (!wait_bounded(&sm.r_free[bi], ph ^ 1u, abort_flag, p.status, 2, p.wait_limit)) break;
       sm.r_ring[bi][i] = r;
       tc_fence_before();
       mbar_arrive(&sm.p_full[bi]);
@@ -339,61 +441,83 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     sm.rcp[i] = __frcp_rn(d);
     mbar_arrive(&sm.done);
   } else if (warp < 8) {
-    // ------------------------------------------------ PV / output owners
+    // ------------------------------------------------------ output owners
     const int i = threadIdx.x - 128;
     const uint32_t lane_addr = tmem + ((uint32_t)((warp - 4) * 32) << 16);
-    float RO[D];
-#pragma unroll
-    for (int c = 0; c < D; ++c) RO[c] = 0.0f;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
       const uint32_t ph = (t >> 1) & 1;
-      if (!wait_bounded(&sm.p_full[bi], ph, abort_flag, p.status, 3)) break;
+      if (!wait_bounded(&sm.p_full[bi], ph, abort_flag, p.status, 3, p.wait_limit)) break;
       const float r = sm.r_ring[bi][i];
       mbar_arrive(&sm.r_free[bi]);
-      if (r != 1.0f) {
+      // RO *= r (exact no-op where r == 1; nothing to scale before tile 0).
+      // Waiting for the previous tile's identity MMAs also keeps ro_ready at
+      // most one phase ahead of the MMA issuer's wait on it.
+      if (t > 0 && !wait_bounded(&sm.id_done, (uint32_t)((t - 1) & 1), abort_flag, p.status, 15, p.wait_limit)) break;
+      if (t > 0 && __any_sync(0xffffffffu, r != 1.0f)) {
+        tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D; ++c) RO[c] = __fmul_rn(RO[c], r);
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t v[32];
+          tmem_ld32(lane_addr + kColRO + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), r));
+          tmem_st32(lane_addr + kColRO + c0, v);
+        }
+        tmem_wait_st();
       }
+      tc_fence_before();
+      mbar_arrive(&sm.ro_ready);
+      // repack each FP16 K32 buffer in place: one value per column -> two
+      // per column (the FP16 A-operand layout of the identity MMAs)
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
-        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4)) {
+        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
           ok = false;
           break;
         }
         tc_fence_after();
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 64) {
-          uint32_t hv[32];
-          tmem_ld64_f16(lane_addr + kColO + 128 * sl + c0, hv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            RO[c0 + 2 * j] = add_f16(RO[c0 + 2 * j], (uint16_t)(hv[j] & 0xFFFFu));
-            RO[c0 + 2 * j + 1] = add_f16(RO[c0 + 2 * j + 1], (uint16_t)(hv[j] >> 16));
-          }
-        }
+        const uint32_t ob = lane_addr + kColO + 128 * sl;
+        uint32_t h0[32], h1[32];
+        tmem_ld32_pack16(ob, h0);
+        if (D == 128) tmem_ld32_pack16(ob + 64, h1);
+        tmem_wait_ld();
+        tmem_st32(ob, h0);
+        if (D == 128) tmem_st32(ob + 32, h1);
+        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.o_free[sl]);
+        mbar_arrive(&sm.o_packed[sl]);
       }
     }
-    if (wait_bounded(&sm.done, 0, abort_flag, p.status, 5) && !*abort_flag) {
+    // epilogue: RO after the last identity MMAs, then 1/d, V scale, BF16
+    if (ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) &&
+        wait_bounded(&sm.id_done, (uint32_t)((T - 1) & 1), abort_flag, p.status, 16, p.wait_limit) && !*abort_flag) {
+      tc_fence_after();
       const int row = qt * kQTile + i;
       const float rc = sm.rcp[i];
-      if (row < p.N) {
-        const float* vs = p.v_scale + (size_t)bh * D;
-        uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h;
+      const float* vs = p.v_scale + (size_t)bh * D;
+      uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h;
 #pragma unroll
-        for (int c = 0; c < D; c += 8) {
-          uint32_t w[4];
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(lane_addr + kColRO + c0, v);
+        tmem_wait_ld();
+        if (row < p.N) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t lo = f32_to_bf16_rn(__fmul_rn(__fmul_rn(RO[c + 2 * e], rc), vs[c + 2 * e]));
-            const uint32_t hi = f32_to_bf16_rn(__fmul_rn(__fmul_rn(RO[c + 2 * e + 1], rc), vs[c + 2 * e + 1]));
-            w[e] = lo | (hi << 16);
+          for (int c = 0; c < 32; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int cc = c0 + c + 2 * e;
+              const uint32_t lo = f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e]), rc), vs[cc]));
+              const uint32_t hi =
+                  f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e + 1]), rc), vs[cc + 1]));
+              w[e] = lo | (hi << 16);
+            }
+            *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-          *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
@@ -405,59 +529,85 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
       for (int t = 0; t < T; ++t) {
         const int st = t % kStages;
-        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag, p.status, 6))
+        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag, p.status, 6, p.wait_limit))
           break;
+        if (t == p.stall_tile) continue;  // test hook: this tile never arrives
         mbar_expect_tx(&sm.kv_full[st], 2 * kKTile * D);
         tma_load_3d(sm.k[st], &tm_k, 0, t * kKTile, bh, &sm.kv_full[st]);
         tma_load_3d(sm.v[st], &tm_v, t * kKTile, 0, bh, &sm.kv_full[st]);
         issued = t + 1;
       }
       // leave no copy in flight: wait for every issued stage and for Q
-      wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, false);
+      wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
       for (int u = max(0, issued - kStages); u < issued; ++u)
-        wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8, false);
+        if (u != p.stall_tile)
+          wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8,
+                       p.wait_limit, false);
     }
   } else {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>();
-      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9);
+      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>(), iid = idesc_id();
       const uint64_t qdesc = smem_desc(sm.q, D);
-      for (int t = 0; ok && t <= T; ++t) {
-        if (t < T) {
-          const int st = t % kStages, bi = t & 1;
-          if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10)) break;
-          if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11)) break;
-          tc_fence_after();
-          const uint64_t kdesc = smem_desc(sm.k[st], D);
+      const uint64_t idn = smem_desc_noswz(sm.ident, 128, 256);
+      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
+      // QK(t) into score buffer t % 2
+      auto issue_qk = [&](int t) -> bool {
+        const int st = t % kStages, bi = t & 1;
+        if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit)) return false;
+        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit)) return false;
+        tc_fence_after();
+        const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk)
-            mma_i8_ss(tmem + kColS + 64 * bi, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
-          tc_commit(&sm.s_full[bi]);
-        }
-        if (t >= 1) {
-          const int u = t - 1, bu = u & 1, su = u % kStages;
-          if (!wait_bounded(&sm.p_full[bu], (uint32_t)((u >> 1) & 1), abort_flag, p.status, 12)) break;
-          tc_fence_after();
-          const uint64_t vdesc = smem_desc(sm.v[su], kKTile);
+        for (int kk = 0; kk < D / 32; ++kk)
+          mma_i8_ss(tmem + kColS + 64 * bi, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
+        tc_commit(&sm.s_full[bi]);
+        return true;
+      };
+      if (ok && T > 0) ok = issue_qk(0);
+      if (ok && T > 1) ok = issue_qk(1);
+      for (int u = 0; ok && u < T; ++u) {
+        const int bu = u & 1, su = u % kStages;
+        // PV(u): two K32 slices, each into its own FP16 buffer from zero
+        if (!wait_bounded(&sm.p_full[bu], (uint32_t)((u >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
+        tc_fence_after();
+        const uint64_t vdesc = smem_desc(sm.v[su], kKTile);
 #pragma unroll
-          for (int sl = 0; sl < 2; ++sl) {
-            if (!wait_bounded(&sm.o_free[sl], (uint32_t)((u & 1) ^ 1), abort_flag, p.status, 13)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            mma_f8_ts(tmem + kColO + 128 * sl, tmem + kColS + 64 * bu + 8 * sl, vdesc + 2 * sl, ipv, 0);
-            tc_commit(&sm.o_full[sl]);
+        for (int sl = 0; sl < 2; ++sl) {
+          if (!wait_bounded(&sm.o_free[sl], (uint32_t)((u & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
-          tc_commit(&sm.kv_empty[su]);
-          tc_commit(&sm.s_free[bu]);
+          tc_fence_after();
+          mma_f8_ts(tmem + kColO + 128 * sl, tmem + kColS + 64 * bu + 8 * sl, vdesc + 2 * sl, ipv, 0);
+          tc_commit(&sm.o_full[sl]);
         }
+        if (!ok) break;
+        tc_commit(&sm.kv_empty[su]);
+        tc_commit(&sm.s_free[bu]);
+        // QK(u+2) into the score buffer PV(u) just read
+        if (u + 2 < T && !(ok = issue_qk(u + 2))) break;
+        // RO += float(buffer) per slice, in slice order, after the rescale
+        if (!wait_bounded(&sm.ro_ready, (uint32_t)(u & 1), abort_flag, p.status, 17, p.wait_limit)) break;
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          if (!wait_bounded(&sm.o_packed[sl], (uint32_t)(u & 1), abort_flag, p.status, 18, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int blk = 0; blk < D / 16; ++blk)
+            mma_f16_ts(tmem + kColRO + 16 * blk, tmem + kColO + 128 * sl + 8 * blk, idn, iid,
+                       (u > 0 || sl > 0) ? 1u : 0u);
+          tc_commit(&sm.o_free[sl]);
+        }
+        if (!ok) break;
+        tc_commit(&sm.id_done);
       }
       // no MMA may still be writing TMEM when it is freed
       tc_commit(&sm.drain);
-      wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, false);
+      wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
     __syncwarp();
   }
@@ -494,12 +644,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
     mbar_expect_tx(&sm.kv_full[0], kKTile * D);
     tma_load_3d(sm.k[0], &tm_k, 0, kt * kKTile, bh, &sm.kv_full[0]);
-    wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, false);
-    wait_bounded(&sm.kv_full[0], 0, abort_flag, nullptr, 8, false);
+    wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
+    wait_bounded(&sm.kv_full[0], 0, abort_flag, nullptr, 8, p.wait_limit, false);
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9) &&
-                wait_bounded(&sm.kv_full[0], 0, abort_flag, p.status, 10);
+      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit) &&
+                wait_bounded(&sm.kv_full[0], 0, abort_flag, p.status, 10, p.wait_limit);
       if (ok) {
         tc_fence_after();
         const uint64_t qdesc = smem_desc(sm.q, D), kdesc = smem_desc(sm.k[0], D);
@@ -508,11 +658,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           mma_i8_ss(tmem + kColS, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk(), kk > 0);
       }
       tc_commit(&sm.s_full[0]);
-      wait_bounded(&sm.s_full[0], 0, abort_flag, nullptr, 14, false);
+      wait_bounded(&sm.s_full[0], 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
     __syncwarp();
   } else if (warp < 4) {
-    if (wait_bounded(&sm.s_full[0], 0, abort_flag, p.status, 1) && !*abort_flag) {
+    if (wait_bounded(&sm.s_full[0], 0, abort_flag, p.status, 1, p.wait_limit) && !*abort_flag) {
       tc_fence_after();
       uint32_t S[64];
       tmem_ld64(tmem + ((uint32_t)(warp * 32) << 16) + kColS, S);

@@ -15,6 +15,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 int g_mainloop = SAGE_MAINLOOP_DEFAULT;
 bool g_mainloop_env_read = false;
+int g_stall_tile = -1;                        // test hook (sage_debug_set_stall)
+long long g_wait_limit = kDefaultWaitLimit;
 
 struct Dims {
   int B, N, H, D, Nq, Nk, G32, T64;
@@ -135,6 +137,8 @@ AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const i
   p.Nq = d.Nq; p.Nk = d.Nk; p.G32 = d.G32; p.T64 = d.T64;
   p.sl2 = log2_scale(sm_scale, d.D);
   p.status = static_cast<DeviceStatus*>(ws);
+  p.wait_limit = g_wait_limit;
+  p.stall_tile = g_stall_tile;
   return p;
 }
 
@@ -285,6 +289,12 @@ int sage_set_mainloop(int which) {
 }
 
 int sage_get_mainloop(void) { return resolved_mainloop(); }
+
+int sage_debug_set_stall(int k_tile, long long wait_limit_cycles) {
+  g_stall_tile = k_tile < 0 ? -1 : k_tile;
+  g_wait_limit = wait_limit_cycles > 0 ? wait_limit_cycles : kDefaultWaitLimit;
+  return SAGE_OK;
+}
 
 int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int H, int D, int b,
                       int h, int q_tile, int k_tile, int32_t* s_out, void* workspace,

@@ -35,7 +35,11 @@ struct AttnParams {
   int Nq, Nk, G32, T64;
   float sl2;             // fl32(sm_scale * log2 e)
   DeviceStatus* status;
+  long long wait_limit;  // clock cycles a bounded device wait may spin
+  int stall_tile;        // test hook: the producer withholds this K/V tile (-1: none)
 };
+
+constexpr long long kDefaultWaitLimit = 2000000000LL;  // ~1 s at 1.9 GHz
 
 // --------------------------------------------------------------- numerics
 // Pack two floats into two E4M3 bytes (round to nearest even, satfinite);

@@ -167,6 +167,15 @@ SAGE_API const char* sage_strerror(int code);
 SAGE_API int sage_set_mainloop(int which);
 SAGE_API int sage_get_mainloop(void);
 
+/* Test export for failure detection.  From the next call on, the tcgen05
+ * mainloop's producer withholds K/V tile `k_tile` of every CTA (< 0: none),
+ * and every bounded device wait gives up after `wait_limit_cycles` SM clock
+ * cycles (<= 0: the default, about one second).  A withheld tile makes the
+ * waits run out: the kernel records SAGE_ERR_TIMEOUT in the status word,
+ * abandons the work, frees its tensor memory and returns, leaving the
+ * context usable.  Process-wide; call with (-1, 0) to restore. */
+SAGE_API int sage_debug_set_stall(int k_tile, long long wait_limit_cycles);
+
 /* Size of the fixed device array behind sage_attn_fwd_noalloc (64 MiB). */
 #define SAGE_NOALLOC_SCRATCH_BYTES (64u << 20)
 

@@ -36,7 +36,9 @@ def run_fwd(sage, q, k, v, mainloop, sm_scale=0.0, out=None):
         out = torch.empty((B, N, H, D), dtype=torch.bfloat16, device=q.device)
     sage.sage_attn_fwd(q, k, v, out, sm_scale, ws)
     st = sage.sage_read_device_status(ws)
-    assert st == sage.SAGE_OK, sage.sage_strerror(st)
+    if st != sage.SAGE_OK:
+        code, where, block = ws[:12].view(torch.int32).tolist()
+        raise AssertionError(f"{sage.sage_strerror(st)} (wait {where}, block {block})")
     return out, ws
 
 

@@ -1,0 +1,44 @@
+"""Failure detection on the GPU without a fault: the tcgen05 producer is
+told to withhold one K/V tile, so the bounded waits behind it run out after
+a short limit.  The kernel must report SAGE_ERR_TIMEOUT through the status
+word, abandon the work, free its tensor memory and return; the next call on
+the same context must succeed and match the oracle."""
+import numpy as np
+import pytest
+
+import gpu_util as gu
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+torch = pytest.importorskip("torch")
+
+
+def test_withheld_tile_times_out_and_context_survives():
+    import fp8_quantized_exact_b200 as sage
+    from fp8_quantized_exact_b200 import build
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    dev = torch.device("cuda:0")
+    sage.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT)
+    if sage.sage_get_mainloop() != sage.SAGE_MAINLOOP_TCGEN05:
+        pytest.skip("the bounded waits live in the tcgen05 mainloop")
+    inp = synth.custom(1, 700, 2, 128, seed=4)
+    (q, k, v), _ = gu.to_device(inp, dev)
+    B, N, H, D = q.shape
+    ws = sage.workspace(sage.SAGE_OP_ATTN_FWD, B, N, H, D, dev)
+    out = torch.empty_like(q)
+    try:
+        sage.sage_debug_set_stall(3, 2_000_000)  # about 1 ms per wait
+        sage.sage_attn_fwd(q, k, v, out, 0.0, ws)
+        st = sage.sage_read_device_status(ws)
+        code, where, block = ws[:12].view(torch.int32).tolist()
+    finally:
+        sage.sage_debug_set_stall(-1, 0)
+    assert st == sage.SAGE_ERR_TIMEOUT and code == st, (st, where, block)
+    assert where > 0 and 0 <= block < (N + 127) // 128 * H * B
+    # the context is still usable and the next call is correct
+    out2, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05)
+    qz = oracle.quantize(inp.q, inp.k, inp.v)
+    gu.compare_out(out2.float().cpu().numpy(), oracle.bf16_bits_to_float(oracle.attention(qz)), "after timeout")

@@ -143,6 +143,25 @@ class ClockSampler:
                 "samples": len(rows), "reasons": sorted(reasons)}
 
 
+# ------------------------------------------------------------ multi-rank
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (the job's time is its slowest
+    rank's); a no-op for one rank.  Timing plumbing only: no data crosses."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Throughput of all ranks together: every rank runs its own replica of
+    the workload, so the job does world * ops in the slowest rank's time."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------- reference
 def cpu_sample(cfg, inp, groups: int):
     """Time the oracle on a bounded sample of the workload and extrapolate the
@@ -289,14 +308,10 @@ def main():
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
-    total_ms = t0.elapsed_time(t1)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ml_ms = [a.elapsed_time(b) for a, b in evs]
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
     ms_step = total_ms / args.steps
-    value = world * cfg.ops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tops(cfg.ops, world, ms_step)
     ml_avg = statistics.mean(ml_ms)
 
     # end to end through the public call with pinned host buffers
@@ -320,11 +335,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
     st = sage.sage_read_device_status(ws_f)
     if st != sage.SAGE_OK:
         raise RuntimeError(f"device status after e2e: {sage.sage_strerror(st)}")
@@ -349,7 +360,7 @@ def main():
                                         "(dense INT8/FP8 : BF16 nominal ratio), burst",
                          "kernel": f"attn mainloop ({ml_name})",
                          "traffic": recorded_traffic(cfg.name, ml_name)},
-            "e2e": {"value": cfg.ops / (e2e_ms * 1e-3) / 1e12 * world, "unit": UNIT,
+            "e2e": {"value": whole_job_tops(cfg.ops, world, e2e_ms), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * 8,
             "clocks": clk.summary(),

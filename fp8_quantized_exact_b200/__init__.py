@@ -190,7 +190,7 @@ def sage_attn_fwd_noalloc(q, k, v, out, sm_scale, stream=None):
     _check(lib().sage_attn_fwd_noalloc(_view(q), _view(k), _view(v), _ptr(out), out.stride(0),
                                        out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
                                        _stream(stream)),
-           "sage_attn_fwd_noalloc", "sage_debug_set_stall")
+           "sage_attn_fwd_noalloc")
 
 
 def sage_read_device_status(workspace, stream=None) -> int:

@@ -42,9 +42,9 @@
 namespace sage {
 namespace {
 
-constexpr int kThreadsTC = 320;
-constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kThreadsTC = 448;
+constexpr int kLoadWarp = 12;
+constexpr int kMmaWarp = 13;
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
@@ -239,6 +239,16 @@ __device__ __forceinline__ void tmem_ld32_pack16(uint32_t taddr, uint32_t (&r)[3
                : "r"(taddr));
 }
 
+// 32 columns of FP16 values -> 16 registers, two per register.
+__device__ __forceinline__ void tmem_ld16_pack16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.pack::16b.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // FP16 x FP16 -> FP32 MMA with A in TMEM (M = 128).
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                            uint32_t accumulate) {
@@ -360,6 +370,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  constexpr int DH = D / 2;  // output columns owned by one output thread
   TcSmem<D>& sm = tc_smem<D>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -377,27 +388,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_free[i], 1);
       mbar_init(&sm.p_full[i], kQTile);
-      mbar_init(&sm.r_free[i], kQTile);
+      mbar_init(&sm.r_free[i], 2 * kQTile);
       mbar_init(&sm.o_full[i], 1);
-      mbar_init(&sm.o_packed[i], kQTile);
-      mbar_init(&sm.o_free[i], 1);
+      mbar_init(&sm.o_free[i], 2 * kQTile);
     }
-    mbar_init(&sm.ro_ready, kQTile);
-    mbar_init(&sm.id_done, 1);
     mbar_init(&sm.done, kQTile);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == kLoadWarp) {
-    // FP16 identity in the no-swizzle K-major layout: element (n, k) at
-    // (n/8)*256 + (k/8)*128 + (n%8)*16 + (k%8)*2 bytes
-    for (int e = lane; e < 256; e += 32) {
-      const int n = e >> 4, k = e & 15;
-      sm.ident[((n >> 3) * 256 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) / 2] =
-          (n == k) ? (uint16_t)0x3C00u : (uint16_t)0u;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
@@ -440,10 +438,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     sm.rcp[i] = __frcp_rn(d);
     mbar_arrive(&sm.done);
-  } else if (warp < 8) {
-    // ------------------------------------------------------ output owners
-    const int i = threadIdx.x - 128;
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+  } else if (warp < 12) {
+    // ---------------------------------------- output owners (half rows)
+    const int i = (warp & 3) * 32 + lane;      // row within the tile
+    const int c_base = warp < 8 ? 0 : DH;      // this thread's output columns
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    float RO[DH];
+#pragma unroll
+    for (int c = 0; c < DH; ++c) RO[c] = 0.0f;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
@@ -451,27 +453,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       if (!wait_bounded(&sm.p_full[bi], ph, abort_flag, p.status, 3, p.wait_limit)) break;
       const float r = sm.r_ring[bi][i];
       mbar_arrive(&sm.r_free[bi]);
-      // RO *= r (exact no-op where r == 1; nothing to scale before tile 0).
-      // Waiting for the previous tile's identity MMAs also keeps ro_ready at
-      // most one phase ahead of the MMA issuer's wait on it.
-      if (t > 0 && !wait_bounded(&sm.id_done, (uint32_t)((t - 1) & 1), abort_flag, p.status, 15, p.wait_limit)) break;
-      if (t > 0 && __any_sync(0xffffffffu, r != 1.0f)) {
-        tc_fence_after();
+      if (r != 1.0f) {
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld32(lane_addr + kColRO + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), r));
-          tmem_st32(lane_addr + kColRO + c0, v);
+        for (int c = 0; c < DH; c += 2) {
+          asm("{.reg .b64 a, s; mov.b64 a, {%0, %1}; mov.b64 s, {%2, %2}; mul.rn.f32x2 a, a, s;"
+              " mov.b64 {%0, %1}, a;}"
+              : "+f"(RO[c]), "+f"(RO[c + 1])
+              : "f"(r));
         }
-        tmem_wait_st();
       }
-      tc_fence_before();
-      mbar_arrive(&sm.ro_ready);
-      // repack each FP16 K32 buffer in place: one value per column -> two
-      // per column (the FP16 A-operand layout of the identity MMAs)
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
         if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
@@ -479,45 +469,41 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t ob = lane_addr + kColO + 128 * sl;
-        uint32_t h0[32], h1[32];
-        tmem_ld32_pack16(ob, h0);
-        if (D == 128) tmem_ld32_pack16(ob + 64, h1);
+        uint32_t hv[DH / 2];
+        if (DH == 64) {
+          tmem_ld32_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[32]>(hv));
+        } else {
+          tmem_ld16_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[16]>(hv));
+        }
         tmem_wait_ld();
-        tmem_st32(ob, h0);
-        if (D == 128) tmem_st32(ob + 32, h1);
-        tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.o_packed[sl]);
+        mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
+        // RO += float(tmp), one rounding per element (tmp is exact in FP32)
+#pragma unroll
+        for (int j = 0; j < DH / 2; ++j) {
+          asm("{.reg .b16 lo, hi; mov.b32 {lo, hi}, %2; add.rn.f32.f16 %0, lo, %0;"
+              " add.rn.f32.f16 %1, hi, %1;}"
+              : "+f"(RO[2 * j]), "+f"(RO[2 * j + 1])
+              : "r"(hv[j]));
+        }
       }
     }
-    // epilogue: RO after the last identity MMAs, then 1/d, V scale, BF16
-    if (ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) &&
-        wait_bounded(&sm.id_done, (uint32_t)((T - 1) & 1), abort_flag, p.status, 16, p.wait_limit) && !*abort_flag) {
-      tc_fence_after();
+    if (ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) && !*abort_flag) {
       const int row = qt * kQTile + i;
       const float rc = sm.rcp[i];
-      const float* vs = p.v_scale + (size_t)bh * D;
-      uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h;
+      if (row < p.N) {
+        const float* vs = p.v_scale + (size_t)bh * D + c_base;
+        uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h + c_base;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(lane_addr + kColRO + c0, v);
-        tmem_wait_ld();
-        if (row < p.N) {
+        for (int c = 0; c < DH; c += 8) {
+          uint32_t w[4];
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int cc = c0 + c + 2 * e;
-              const uint32_t lo = f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e]), rc), vs[cc]));
-              const uint32_t hi =
-                  f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e + 1]), rc), vs[cc + 1]));
-              w[e] = lo | (hi << 16);
-            }
-            *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t lo = f32_to_bf16_rn(__fmul_rn(__fmul_rn(RO[c + 2 * e], rc), vs[c + 2 * e]));
+            const uint32_t hi = f32_to_bf16_rn(__fmul_rn(__fmul_rn(RO[c + 2 * e + 1], rc), vs[c + 2 * e + 1]));
+            w[e] = lo | (hi << 16);
           }
+          *reinterpret_cast<uint4*>(dst + c) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
     }
@@ -529,7 +515,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
       for (int t = 0; t < T; ++t) {
         const int st = t % kStages;
-        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag, p.status, 6, p.wait_limit))
+        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag, p.status, 6,
+                          p.wait_limit))
           break;
         if (t == p.stall_tile) continue;  // test hook: this tile never arrives
         mbar_expect_tx(&sm.kv_full[st], 2 * kKTile * D);
@@ -547,15 +534,16 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   } else {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>(), iid = idesc_id();
+      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>();
       const uint64_t qdesc = smem_desc(sm.q, D);
-      const uint64_t idn = smem_desc_noswz(sm.ident, 128, 256);
       bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
       // QK(t) into score buffer t % 2
       auto issue_qk = [&](int t) -> bool {
         const int st = t % kStages, bi = t & 1;
-        if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit)) return false;
-        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit)) return false;
+        if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
+          return false;
+        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit))
+          return false;
         tc_fence_after();
         const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
@@ -587,23 +575,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tc_commit(&sm.s_free[bu]);
         // QK(u+2) into the score buffer PV(u) just read
         if (u + 2 < T && !(ok = issue_qk(u + 2))) break;
-        // RO += float(buffer) per slice, in slice order, after the rescale
-        if (!wait_bounded(&sm.ro_ready, (uint32_t)(u & 1), abort_flag, p.status, 17, p.wait_limit)) break;
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          if (!wait_bounded(&sm.o_packed[sl], (uint32_t)(u & 1), abort_flag, p.status, 18, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int blk = 0; blk < D / 16; ++blk)
-            mma_f16_ts(tmem + kColRO + 16 * blk, tmem + kColO + 128 * sl + 8 * blk, idn, iid,
-                       (u > 0 || sl > 0) ? 1u : 0u);
-          tc_commit(&sm.o_free[sl]);
-        }
-        if (!ok) break;
-        tc_commit(&sm.id_done);
       }
       // no MMA may still be writing TMEM when it is freed
       tc_commit(&sm.drain);

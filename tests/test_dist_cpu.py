@@ -1,0 +1,62 @@
+"""The N > 1 bench path on CPU with two gloo ranks: every rank times its own
+replica and the job reports the slowest rank's time; the reference arm runs
+on rank 0 only."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = 10.0 + 5.0 * rank          # rank 1 is the slow one
+        slow = bench.max_over_ranks(ms, world)
+        out[rank] = (slow, bench.whole_job_tops(1e12, world, slow))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_max_and_aggregate():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_worker, args=(2, _free_port(), out), nprocs=2, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0] == res[1]
+    slow, tops = res[0]
+    assert slow == 15.0
+    assert abs(tops - 2 * 1e12 / 15e-3 / 1e12) < 1e-9
+
+
+def test_reference_arm_runs_on_rank_zero_only(tmp_path):
+    """Under a two-rank launch the reference arm prints from rank 0 and the
+    other rank exits 0 without work (small config, one step)."""
+    env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", env["MASTER_PORT"],
+           os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "small",
+           "--steps", "1", "--warmup", "0", "--gpus", "2"]
+    r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and '"impl": "reference"' in lines[0]

@@ -478,11 +478,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
-        // RO += float(tmp), one rounding per element (tmp is exact in FP32)
+        // RO += float(tmp), one rounding per element (float(tmp) is exact):
+        // widen the FP16 pair, then one packed FP32x2 add
 #pragma unroll
         for (int j = 0; j < DH / 2; ++j) {
-          asm("{.reg .b16 lo, hi; mov.b32 {lo, hi}, %2; add.rn.f32.f16 %0, lo, %0;"
-              " add.rn.f32.f16 %1, hi, %1;}"
+          asm("{.reg .b16 lo, hi; .reg .f32 a, b; .reg .b64 x, y;"
+              " mov.b32 {lo, hi}, %2; cvt.f32.f16 a, lo; cvt.f32.f16 b, hi;"
+              " mov.b64 x, {a, b}; mov.b64 y, {%0, %1}; add.rn.f32x2 y, y, x; mov.b64 {%0, %1}, y;}"
               : "+f"(RO[2 * j]), "+f"(RO[2 * j + 1])
               : "r"(hv[j]));
         }

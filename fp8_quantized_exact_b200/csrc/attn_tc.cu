@@ -48,8 +48,7 @@ constexpr int kMmaWarp = 13;
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
-constexpr uint32_t kColRO = 128;   // FP32 output accumulator of columns [0, D/2)
-constexpr uint32_t kColPk = 192;   // two packed FP16 copies of columns [0, D/2) of a K32 buffer
+constexpr uint32_t kColRO = 128;   // FP32 output accumulator, D columns
 constexpr uint32_t kColO = 256;    // two FP16 PV buffers of 128 columns (one per K32 slice)
 
 template <int D>
@@ -64,7 +63,7 @@ struct TcSmem {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_full[2], o_free[2];
+  uint64_t o_full[2], o_packed[2], o_free[2];
   uint64_t ro_ready, id_done;
   uint64_t done, drain;
   uint32_t tmem_base;
@@ -371,8 +370,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  constexpr int DA = D / 2;      // columns accumulated by identity MMAs into TMEM
-  constexpr int DB = D - DA;     // columns accumulated in registers
+  constexpr int DH = D / 2;  // output columns owned by one output thread
   TcSmem<D>& sm = tc_smem<D>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -394,22 +392,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_free[i], 2 * kQTile);
     }
-    mbar_init(&sm.ro_ready, kQTile);
-    mbar_init(&sm.id_done, 1);
     mbar_init(&sm.done, kQTile);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == kLoadWarp) {
-    // FP16 16x16 identity in the no-swizzle K-major layout: element (n, k) at
-    // (n/8)*256 + (k/8)*128 + (n%8)*16 + (k%8)*2 bytes
-    for (int e = lane; e < 256; e += 32) {
-      const int n = e >> 4, k = e & 15;
-      sm.ident[((n >> 3) * 256 + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2) / 2] =
-          (n == k) ? (uint16_t)0x3C00u : (uint16_t)0u;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
@@ -452,98 +438,14 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     sm.rcp[i] = __frcp_rn(d);
     mbar_arrive(&sm.done);
-  } else if (warp < 8) {
-    // ------------------ output owners, columns [0, DA): RO in TMEM, added by MMA
-    const int i = threadIdx.x - 128;
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    bool ok = true;
-    for (int t = 0; t < T && ok; ++t) {
-      const int bi = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      if (!wait_bounded(&sm.p_full[bi], ph, abort_flag, p.status, 3, p.wait_limit)) break;
-      const float r = sm.r_ring[bi][i];
-      mbar_arrive(&sm.r_free[bi]);
-      // take columns [0, DA) of both FP16 buffers into registers first, so
-      // that the buffers are released without waiting for any identity MMA
-      uint32_t hv[2][DA / 2];
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (DA == 64) tmem_ld32_pack16(lane_addr + kColO + 128 * sl, *reinterpret_cast<uint32_t(*)[32]>(hv[sl]));
-        else tmem_ld16_pack16(lane_addr + kColO + 128 * sl, *reinterpret_cast<uint32_t(*)[16]>(hv[sl]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sm.o_free[sl]);
-      }
-      if (!ok) break;
-      // after the identity MMAs of tile t-1: RO *= r (exact no-op where
-      // r == 1; nothing to scale before tile 0), then the packed FP16 copies
-      // (two values per column) that the identity MMAs of tile t read.  The
-      // wait also keeps ro_ready at most one phase ahead of its consumer.
-      if (t > 0 && !wait_bounded(&sm.id_done, (uint32_t)((t - 1) & 1), abort_flag, p.status, 15, p.wait_limit))
-        break;
-      tc_fence_after();
-      if (t > 0 && __any_sync(0xffffffffu, r != 1.0f)) {
-        uint32_t v[32];
-#pragma unroll
-        for (int c0 = 0; c0 < DA; c0 += 32) {
-          tmem_ld32(lane_addr + kColRO + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__fmul_rn(__uint_as_float(v[j]), r));
-          tmem_st32(lane_addr + kColRO + c0, v);
-        }
-      }
-#pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        if (DA == 64) tmem_st32(lane_addr + kColPk + 32 * sl, *reinterpret_cast<uint32_t(*)[32]>(hv[sl]));
-        else tmem_st16(lane_addr + kColPk + 32 * sl, *reinterpret_cast<uint32_t(*)[16]>(hv[sl]));
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.ro_ready);
-    }
-    if (ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) &&
-        wait_bounded(&sm.id_done, (uint32_t)((T - 1) & 1), abort_flag, p.status, 16, p.wait_limit) &&
-        !*abort_flag) {
-      tc_fence_after();
-      const int row = qt * kQTile + i;
-      const float rc = sm.rcp[i];
-      const float* vs = p.v_scale + (size_t)bh * D;
-      uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h;
-#pragma unroll
-      for (int c0 = 0; c0 < DA; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(lane_addr + kColRO + c0, v);
-        tmem_wait_ld();
-        if (row < p.N) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int cc = c0 + c + 2 * e;
-              const uint32_t lo = f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e]), rc), vs[cc]));
-              const uint32_t hi =
-                  f32_to_bf16_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[c + 2 * e + 1]), rc), vs[cc + 1]));
-              w[e] = lo | (hi << 16);
-            }
-            *reinterpret_cast<uint4*>(dst + c0 + c) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
-      }
-    }
   } else if (warp < 12) {
-    // ------------- output owners, columns [DA, D): RO in registers
+    // ---------------------------------------- output owners (half rows)
     const int i = (warp & 3) * 32 + lane;      // row within the tile
+    const int c_base = warp < 8 ? 0 : DH;      // this thread's output columns
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    float RO[DB];
+    float RO[DH];
 #pragma unroll
-    for (int c = 0; c < DB; ++c) RO[c] = 0.0f;
+    for (int c = 0; c < DH; ++c) RO[c] = 0.0f;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
@@ -553,7 +455,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_arrive(&sm.r_free[bi]);
       if (r != 1.0f) {
 #pragma unroll
-        for (int c = 0; c < DB; c += 2) {
+        for (int c = 0; c < DH; c += 2) {
           asm("{.reg .b64 a, s; mov.b64 a, {%0, %1}; mov.b64 s, {%2, %2}; mul.rn.f32x2 a, a, s;"
               " mov.b64 {%0, %1}, a;}"
               : "+f"(RO[c]), "+f"(RO[c + 1])
@@ -567,16 +469,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           break;
         }
         tc_fence_after();
-        uint32_t hv[DB / 2];
-        if (DB == 64) tmem_ld32_pack16(lane_addr + kColO + 128 * sl + DA, *reinterpret_cast<uint32_t(*)[32]>(hv));
-        else tmem_ld16_pack16(lane_addr + kColO + 128 * sl + DA, *reinterpret_cast<uint32_t(*)[16]>(hv));
+        uint32_t hv[DH / 2];
+        if (DH == 64) {
+          tmem_ld32_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[32]>(hv));
+        } else {
+          tmem_ld16_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[16]>(hv));
+        }
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
         // RO += float(tmp), one rounding per element (float(tmp) is exact):
         // widen the FP16 pair, then one packed FP32x2 add
 #pragma unroll
-        for (int j = 0; j < DB / 2; ++j) {
+        for (int j = 0; j < DH / 2; ++j) {
           asm("{.reg .b16 lo, hi; .reg .f32 a, b; .reg .b64 x, y;"
               " mov.b32 {lo, hi}, %2; cvt.f32.f16 a, lo; cvt.f32.f16 b, hi;"
               " mov.b64 x, {a, b}; mov.b64 y, {%0, %1}; add.rn.f32x2 y, y, x; mov.b64 {%0, %1}, y;}"
@@ -589,10 +494,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const int row = qt * kQTile + i;
       const float rc = sm.rcp[i];
       if (row < p.N) {
-        const float* vs = p.v_scale + (size_t)bh * D + DA;
-        uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h + DA;
+        const float* vs = p.v_scale + (size_t)bh * D + c_base;
+        uint16_t* dst = p.out + b * p.os_b + (int64_t)row * p.os_n + h * p.os_h + c_base;
 #pragma unroll
-        for (int c = 0; c < DB; c += 8) {
+        for (int c = 0; c < DH; c += 8) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -631,9 +536,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   } else {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>(), iid = idesc_id();
+      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>();
       const uint64_t qdesc = smem_desc(sm.q, D);
-      const uint64_t idn = smem_desc_noswz(sm.ident, 128, 256);
       bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
       // QK(t) into score buffer t % 2
       auto issue_qk = [&](int t) -> bool {
@@ -648,20 +552,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         for (int kk = 0; kk < D / 32; ++kk)
           mma_i8_ss(tmem + kColS + 64 * bi, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
         tc_commit(&sm.s_full[bi]);
-        return true;
-      };
-      // RO[:, 0:DA) += float(buffer) of tile v, slice by slice, through the
-      // identity: each output column receives exactly one non-zero product
-      auto issue_id = [&](int v) -> bool {
-        if (!wait_bounded(&sm.ro_ready, (uint32_t)(v & 1), abort_flag, p.status, 17, p.wait_limit)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl)
-#pragma unroll
-          for (int blk = 0; blk < DA / 16; ++blk)
-            mma_f16_ts(tmem + kColRO + 16 * blk, tmem + kColPk + 32 * sl + 8 * blk, idn, iid,
-                       (v > 0 || sl > 0) ? 1u : 0u);
-        tc_commit(&sm.id_done);
         return true;
       };
       if (ok && T > 0) ok = issue_qk(0);
@@ -687,10 +577,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         tc_commit(&sm.s_free[bu]);
         // QK(u+2) into the score buffer PV(u) just read
         if (u + 2 < T && !(ok = issue_qk(u + 2))) break;
-        // the identity MMAs of the previous tile (its copies are long done)
-        if (u >= 1 && !(ok = issue_id(u - 1))) break;
       }
-      if (ok && T > 0) issue_id(T - 1);
       // no MMA may still be writing TMEM when it is freed
       tc_commit(&sm.drain);
       wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, p.wait_limit, false);

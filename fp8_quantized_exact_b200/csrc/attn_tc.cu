@@ -61,7 +61,7 @@ struct TcSmem {
   float rcp[kQTile];
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[2];
   uint64_t p_full[2], r_free[2];
   uint64_t o_full[2], o_packed[2], o_free[2];
   uint64_t ro_ready, id_done;
@@ -386,7 +386,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 1);
       mbar_init(&sm.p_full[i], kQTile);
       mbar_init(&sm.r_free[i], 2 * kQTile);
       mbar_init(&sm.o_full[i], 1);
@@ -544,8 +543,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const int st = t % kStages, bi = t & 1;
         if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
           return false;
-        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit))
-          return false;
+        // no wait for PV(t-2), which read its probabilities from this score
+        // buffer: MMAs issued by one thread execute in issue order, so QK(t)
+        // writes the buffer only after PV(t-2) has read it
         tc_fence_after();
         const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
@@ -574,7 +574,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         if (!ok) break;
         tc_commit(&sm.kv_empty[su]);
-        tc_commit(&sm.s_free[bu]);
         // QK(u+2) into the score buffer PV(u) just read
         if (u + 2 < T && !(ok = issue_qk(u + 2))) break;
       }

@@ -42,14 +42,16 @@
 namespace sage {
 namespace {
 
-constexpr int kThreadsTC = 448;
+constexpr int kThreadsTC = 480;
 constexpr int kLoadWarp = 12;
-constexpr int kMmaWarp = 13;
+constexpr int kMmaWarp = 13;   // QK issuer; also allocates and frees the tensor memory
+constexpr int kPvWarp = 14;    // PV issuer
+constexpr int kOBufs = 3;      // ring of FP16 PV buffers (one K32 slice each)
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
 constexpr uint32_t kColRO = 128;   // FP32 output accumulator, D columns
-constexpr uint32_t kColO = 256;    // two FP16 PV buffers of 128 columns (one per K32 slice)
+constexpr uint32_t kColO = 128;    // ring of kOBufs FP16 PV buffers of 128 columns
 
 template <int D>
 struct TcSmem {
@@ -61,11 +63,11 @@ struct TcSmem {
   float rcp[kQTile];
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2];
+  uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_full[2], o_packed[2], o_free[2];
+  uint64_t o_full[kOBufs], o_free[kOBufs];
   uint64_t ro_ready, id_done;
-  uint64_t done, drain;
+  uint64_t done, drain, drain2;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -382,17 +384,21 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+      mbar_init(&sm.kv_empty[s], 2);  // released by both MMA issuers
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_free[i], 1);
       mbar_init(&sm.p_full[i], kQTile);
       mbar_init(&sm.r_free[i], 2 * kQTile);
+    }
+    for (int i = 0; i < kOBufs; ++i) {
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_free[i], 2 * kQTile);
     }
     mbar_init(&sm.done, kQTile);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain2, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -463,20 +469,21 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {
-        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
+        const int k = 2 * t + sl, ob = k % kOBufs;  // position in the buffer ring
+        if (!wait_bounded(&sm.o_full[ob], (uint32_t)((k / kOBufs) & 1), abort_flag, p.status, 4, p.wait_limit)) {
           ok = false;
           break;
         }
         tc_fence_after();
         uint32_t hv[DH / 2];
         if (DH == 64) {
-          tmem_ld32_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[32]>(hv));
+          tmem_ld32_pack16(lane_addr + kColO + 128 * ob + c_base, *reinterpret_cast<uint32_t(*)[32]>(hv));
         } else {
-          tmem_ld16_pack16(lane_addr + kColO + 128 * sl + c_base, *reinterpret_cast<uint32_t(*)[16]>(hv));
+          tmem_ld16_pack16(lane_addr + kColO + 128 * ob + c_base, *reinterpret_cast<uint32_t(*)[16]>(hv));
         }
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
+        mbar_arrive(&sm.o_free[ob]);  // the buffer may be overwritten now
         // RO += float(tmp), one rounding per element (float(tmp) is exact):
         // widen the FP16 pair, then one packed FP32x2 add
 #pragma unroll
@@ -532,54 +539,64 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8,
                        p.wait_limit, false);
     }
-  } else {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------- QK issuer
     if (lane == 0) {
-      const uint32_t iqk = idesc_qk(), ipv = idesc_pv<D>();
+      const uint32_t iqk = idesc_qk();
       const uint64_t qdesc = smem_desc(sm.q, D);
       bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
-      // QK(t) into score buffer t % 2
-      auto issue_qk = [&](int t) -> bool {
+      for (int t = 0; ok && t < T; ++t) {
         const int st = t % kStages, bi = t & 1;
         if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
-          return false;
-        // no wait for PV(t-2), which read its probabilities from this score
-        // buffer: MMAs issued by one thread execute in issue order, so QK(t)
-        // writes the buffer only after PV(t-2) has read it
+          break;
+        // PV(t-2) read its probabilities from this score buffer
+        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit))
+          break;
         tc_fence_after();
         const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
           mma_i8_ss(tmem + kColS + 64 * bi, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
         tc_commit(&sm.s_full[bi]);
-        return true;
-      };
-      if (ok && T > 0) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
-      for (int u = 0; ok && u < T; ++u) {
-        const int bu = u & 1, su = u % kStages;
-        // PV(u): two K32 slices, each into its own FP16 buffer from zero
-        if (!wait_bounded(&sm.p_full[bu], (uint32_t)((u >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
-        tc_fence_after();
-        const uint64_t vdesc = smem_desc(sm.v[su], kKTile);
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          if (!wait_bounded(&sm.o_free[sl], (uint32_t)((u & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_f8_ts(tmem + kColO + 128 * sl, tmem + kColS + 64 * bu + 8 * sl, vdesc + 2 * sl, ipv, 0);
-          tc_commit(&sm.o_full[sl]);
-        }
-        if (!ok) break;
-        tc_commit(&sm.kv_empty[su]);
-        // QK(u+2) into the score buffer PV(u) just read
-        if (u + 2 < T && !(ok = issue_qk(u + 2))) break;
+        tc_commit(&sm.kv_empty[st]);
       }
       // no MMA may still be writing TMEM when it is freed
       tc_commit(&sm.drain);
       wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, p.wait_limit, false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------- PV issuer
+    if (lane == 0) {
+      const uint32_t ipv = idesc_pv<D>();
+      bool ok = true;
+      for (int u = 0; ok && u < T; ++u) {
+        const int bu = u & 1, su = u % kStages;
+        // PV(u): two K32 slices, each into its own FP16 buffer from zero
+        if (!wait_bounded(&sm.p_full[bu], (uint32_t)((u >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
+        // V(u) arrived with K(u) (already waited on by the QK issuer)
+        if (!wait_bounded(&sm.kv_full[su], (uint32_t)((u / kStages) & 1), abort_flag, p.status, 16, p.wait_limit))
+          break;
+        tc_fence_after();
+        const uint64_t vdesc = smem_desc(sm.v[su], kKTile);
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int k = 2 * u + sl, ob = k % kOBufs;
+          if (!wait_bounded(&sm.o_free[ob], (uint32_t)(((k / kOBufs) & 1) ^ 1), abort_flag, p.status, 13,
+                            p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_f8_ts(tmem + kColO + 128 * ob, tmem + kColS + 64 * bu + 8 * sl, vdesc + 2 * sl, ipv, 0);
+          tc_commit(&sm.o_full[ob]);
+        }
+        if (!ok) break;
+        tc_commit(&sm.s_free[bu]);
+        tc_commit(&sm.kv_empty[su]);
+      }
+      tc_commit(&sm.drain2);
+      wait_bounded(&sm.drain2, 0, abort_flag, nullptr, 15, p.wait_limit, false);
     }
     __syncwarp();
   }

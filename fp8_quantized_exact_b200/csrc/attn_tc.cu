@@ -1,28 +1,25 @@
 // Fused attention mainloop on 5th-generation tensor cores (tcgen05, TMEM,
 // TMA), sm_100a.
 //
-// One CTA = one 128-row query tile of one (b, h); ten warps with fixed roles
-// (the ownership split of the pages' VEA-B design, built on TMEM):
-//   warps 0-3  QK/softmax owners: thread i owns query row i (TMEM lane i), its
-//              running max m and denominator d.  Per tile they read the int32
-//              scores from TMEM, scale them, update m, d and the rescale
-//              factor r, and write the E4M3 probabilities back to TMEM.
-//   warps 4-7  output owners: per tile they apply r to the FP32 output row RO
-//              (kept in TMEM) when the max moved, and repack each FP16 K32 PV
-//              buffer in place into the packed FP16 operand layout; at the end
-//              they apply 1/d and the V scale and store BF16.
-//   warp 8     TMA producer: the Q tile once, then K and V^T tiles of 64 keys
-//              into a ring of shared-memory stages.
-//   warp 9     MMA issuer (one thread), per tile: one INT8 QK^T MMA chain into
-//              a TMEM score buffer (two tiles ahead of PV); per K32 slice one
-//              E4M3 MMA, with the probabilities as the TMEM A operand, into an
-//              FP16 accumulator that starts at zero (the instantaneous buffer);
-//              then, per slice, FP16 MMAs of that buffer against a 16x16
-//              identity held in shared memory accumulate it into the FP32 RO.
-//              With one non-zero product per output, each of those adds the
-//              FP16 value exactly to RO with one FP32 rounding in the tensor
-//              core: the ordered "RO += float(tmp)" per slice, done on the
-//              tensor pipe instead of two ALU instructions per element.
+// One CTA = one 128-row query tile of one (b, h); fifteen warps with fixed
+// roles (the ownership split of the pages' VEA-B design, built on TMEM):
+//   warps 0-3   QK/softmax owners: thread i owns query row i (TMEM lane i),
+//               its running max m and denominator d.  Per tile they read the
+//               int32 scores from TMEM, scale them, update m, d and the
+//               rescale factor r, and write the E4M3 probabilities back to
+//               TMEM over the scores they replace.
+//   warps 4-11  output owners: thread (w, lane) owns half of the FP32 output
+//               row RO of row 32*(w%4)+lane in registers.  Per tile it applies
+//               r, then adds each FP16 K32 buffer (read from TMEM) in order;
+//               at the end it applies 1/d and the V scale and stores BF16.
+//   warp 12     TMA producer: the Q tile once, then K and V^T tiles of 64 keys
+//               into a ring of shared-memory stages.
+//   warp 13     QK issuer (one thread): per tile four INT8 MMAs (K = 32 each)
+//               into one of two TMEM score buffers, up to two tiles ahead.
+//   warp 14     PV issuer (one thread): per K32 slice one E4M3 MMA, with the
+//               probabilities as the TMEM A operand, into an FP16 accumulator
+//               that starts at zero (the instantaneous buffer), taken from a
+//               ring of three TMEM buffers.
 // Handoffs are block-scope mbarriers; tcgen05.commit signals MMA completion.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in
 // the status word, raises a CTA-wide abort flag, and every role then leaves
@@ -50,7 +47,6 @@ constexpr int kOBufs = 3;      // ring of FP16 PV buffers (one K32 slice each)
 constexpr int kStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
-constexpr uint32_t kColRO = 128;   // FP32 output accumulator, D columns
 constexpr uint32_t kColO = 128;    // ring of kOBufs FP16 PV buffers of 128 columns
 
 template <int D>
@@ -58,7 +54,6 @@ struct TcSmem {
   alignas(1024) uint8_t q[kQTile * D];
   alignas(1024) uint8_t k[kStages][kKTile * D];
   alignas(1024) uint8_t v[kStages][D * kKTile];
-  alignas(1024) uint16_t ident[16 * 16];  // FP16 16x16 identity, K-major, no swizzle
   float r_ring[2][kQTile];
   float rcp[kQTile];
   uint64_t q_full;
@@ -190,20 +185,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       : "r"(taddr));
 }
 
-// 32 lanes x 64 columns of FP16 (one per 32-bit column) packed two per
-// register: register j holds columns 2j (low half) and 2j+1 (high half).
-__device__ __forceinline__ void tmem_ld64_f16(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.pack::16b.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -224,15 +205,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 #define SAGE_REGS32 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}"
 #define SAGE_REGS32_1 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32}"
 
-// 32 lanes x 32 columns of 32 bits -> 32 registers.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 " SAGE_REGS32 ", [%32];" : SAGE_R32(r) : "r"(taddr));
-}
-// 32 registers -> 32 lanes x 32 columns.
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], " SAGE_REGS32_1 ";" ::"r"(taddr), SAGE_W32(r)
-               : "memory");
-}
 // 64 columns of FP16 values (one per 32-bit column) -> 32 registers, two per
 // register (column 2j in the low half).
 __device__ __forceinline__ void tmem_ld32_pack16(uint32_t taddr, uint32_t (&r)[32]) {
@@ -251,32 +223,6 @@ __device__ __forceinline__ void tmem_ld16_pack16(uint32_t taddr, uint32_t (&r)[1
       : "r"(taddr));
 }
 
-// FP16 x FP16 -> FP32 MMA with A in TMEM (M = 128).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;}" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Descriptor of a K-major tile without swizzle: 8-row x 16-byte core
-// matrices, `lbo` bytes apart along K and `sbo` bytes apart along M/N.
-__device__ __forceinline__ uint64_t smem_desc_noswz(const void* tile, uint32_t lbo, uint32_t sbo) {
-  const uint32_t a = smem_u32(tile);
-  uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1u << 46;
-  return d;  // layout type 0: no swizzle
-}
-
-// Identity MMA: F16 x F16 -> F32, M = 128, N = 16.
-__host__ __device__ constexpr uint32_t idesc_id() {
-  return (1u << 4) | ((uint32_t)(16 >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
-}
-
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -285,17 +231,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// RO + float(h) in one rounding (mixed-precision add; float(h) is exact).
-__device__ __forceinline__ float add_f16(float ro, uint16_t h) {
-  float d;
-  asm("add.rn.f32.f16 %0, %1, %2;" : "=f"(d) : "h"(h), "f"(ro));
-  return d;
-}
-// int32 -> float, exact for |x| < 2^22 (the scores are below 128*127*127).
-__device__ __forceinline__ float i2f_small(int32_t x) {
-  return __fsub_rn(__int_as_float(x + 0x4B400000), 12582912.0f);
-}
-
 __device__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
                "r"(cols)
@@ -565,7 +500,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
     __syncwarp();
-  } else {
+  } else if (warp == kPvWarp) {
     // ------------------------------------------------------- PV issuer
     if (lane == 0) {
       const uint32_t ipv = idesc_pv<D>();

@@ -1,25 +1,29 @@
 // Fused attention mainloop on 5th-generation tensor cores (tcgen05, TMEM,
 // TMA), sm_100a.
 //
-// One CTA = one 128-row query tile of one (b, h); fifteen warps with fixed
+// One CTA = one 128-row query tile of one (b, h); nineteen warps with fixed
 // roles (the ownership split of the pages' VEA-B design, built on TMEM):
-//   warps 0-3   QK/softmax owners: thread i owns query row i (TMEM lane i),
-//               its running max m and denominator d.  Per tile they read the
-//               int32 scores from TMEM, scale them, update m, d and the
-//               rescale factor r, and write the E4M3 probabilities back to
-//               TMEM over the scores they replace.
-//   warps 4-11  output owners: thread (w, lane) owns half of the FP32 output
+//   warps 0-7   QK/softmax owners.  Warp w owns query rows 32*(w%4)..+31
+//               (TMEM lanes of its quadrant) for the 64-key tiles t with
+//               t % 2 == w / 4, so two warps of a quadrant work on
+//               consecutive tiles at once.  Per tile a warp reads the int32
+//               scores from TMEM, takes the tile max, receives the running
+//               max m(t-1) from its partner (shared memory + mbarrier), hands
+//               m(t) on, computes the rescale factor r, the FP32
+//               probabilities, its part of the denominator, and writes the
+//               E4M3 probabilities back to TMEM over the scores.
+//   warps 8-15  output owners: thread (w, lane) owns half of the FP32 output
 //               row RO of row 32*(w%4)+lane in registers.  Per tile it applies
 //               r, then adds each FP16 K32 buffer (read from TMEM) in order;
 //               at the end it applies 1/d and the V scale and stores BF16.
-//   warp 12     TMA producer: the Q tile once, then K and V^T tiles of 64 keys
-//               into a ring of shared-memory stages.
-//   warp 13     QK issuer (one thread): per tile four INT8 MMAs (K = 32 each)
-//               into one of two TMEM score buffers, up to two tiles ahead.
-//   warp 14     PV issuer (one thread): per K32 slice one E4M3 MMA, with the
-//               probabilities as the TMEM A operand, into an FP16 accumulator
-//               that starts at zero (the instantaneous buffer), taken from a
-//               ring of three TMEM buffers.
+//   warp 16     TMA producer: the Q tile once, then K and V^T stages of 128
+//               keys (two tiles) into a ring of shared-memory stages.
+//   warp 17     QK issuer (one thread): per 128-key group four INT8 MMAs
+//               (N = 128, K = 32 each) into one of two TMEM score buffers.
+//   warp 18     PV issuer (one thread): once a tile's probabilities are in,
+//               per K32 slice one E4M3 MMA, with the probabilities as the TMEM
+//               A operand, into an FP16 accumulator that starts at zero (the
+//               instantaneous buffer), one TMEM buffer per slice.
 // Handoffs are block-scope mbarriers; tcgen05.commit signals MMA completion.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in
 // the status word, raises a CTA-wide abort flag, and every role then leaves
@@ -32,6 +36,9 @@
 // FP32 ro_rescale cross from the QK owner to the PV owner; final FP32
 // reciprocal, then V scale, then BF16); the VEA-B role table of the same
 // page; step order from "Sage2 SM89 Temporal Pair Experiment", "Candidate".
+// The denominator is kept as two partial sums, one per softmax warp of a
+// quadrant, each rescaled to the running max of its latest tile and merged
+// at the end; the pages leave its summation order open.
 #include <cuda.h>
 
 #include "sage_common.cuh"
@@ -39,30 +46,34 @@
 namespace sage {
 namespace {
 
-constexpr int kThreadsTC = 480;
-constexpr int kLoadWarp = 12;
-constexpr int kMmaWarp = 13;   // QK issuer; also allocates and frees the tensor memory
-constexpr int kPvWarp = 14;    // PV issuer
-constexpr int kOBufs = 3;      // ring of FP16 PV buffers (one K32 slice each)
-constexpr int kStages = 4;
+constexpr int kThreadsTC = 608;
+constexpr int kLoadWarp = 16;
+constexpr int kQkWarp = 17;    // QK issuer; also allocates and frees the tensor memory
+constexpr int kPvWarp = 18;    // PV issuer
+constexpr int kGroup = 128;    // keys per K/V stage and per QK MMA (two 64-key tiles)
+constexpr int kStages = 3;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // two int32 score buffers of 64 columns (E4M3 P overlays them)
-constexpr uint32_t kColO = 128;    // ring of kOBufs FP16 PV buffers of 128 columns
+constexpr uint32_t kColS = 0;      // two int32 score buffers of 128 columns (one group each); the
+                                   // E4M3 P of a tile overlays the first 16 columns of its 64
+constexpr uint32_t kColO = 256;    // two FP16 PV buffers of 128 columns (one per K32 slice)
 
 template <int D>
 struct TcSmem {
   alignas(1024) uint8_t q[kQTile * D];
-  alignas(1024) uint8_t k[kStages][kKTile * D];
-  alignas(1024) uint8_t v[kStages][D * kKTile];
+  alignas(1024) uint8_t k[kStages][kGroup * D];
+  alignas(1024) uint8_t v[kStages][D * kGroup];
   float r_ring[2][kQTile];
+  float m_x[2][kQTile];               // running max after a tile, for the partner warp
+  float m_fin[2][kQTile], d_fin[2][kQTile];
   float rcp[kQTile];
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_full[kOBufs], o_free[kOBufs];
-  uint64_t ro_ready, id_done;
-  uint64_t done, drain, drain2;
+  uint64_t o_full[2], o_free[2];
+  uint64_t m_full[4][2];
+  uint64_t fin, done;
+  uint64_t drain_qk, drain_pv;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -141,9 +152,9 @@ __device__ __forceinline__ uint64_t smem_desc(const void* tile, int row_bytes) {
 }
 
 // Instruction descriptors: M = 128, K-major A and B.
-// QK: INT8 x INT8 -> S32, N = 64.  PV: E4M3 x E4M3 -> F16, N = D.
-__host__ __device__ constexpr uint32_t idesc_qk() {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKTile >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
+// QK: INT8 x INT8 -> S32, N keys.  PV: E4M3 x E4M3 -> F16, N = D.
+__host__ __device__ constexpr uint32_t idesc_qk(int n) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
 }
 template <int D>
 __host__ __device__ constexpr uint32_t idesc_pv() {
@@ -193,26 +204,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-#define SAGE_R32(r) "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), \
-    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),   \
-    "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),              \
-    "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),              \
-    "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define SAGE_W32(r) "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), \
-    "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),            \
-    "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),          \
-    "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-#define SAGE_REGS32 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}"
-#define SAGE_REGS32_1 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32}"
-
-// 64 columns of FP16 values (one per 32-bit column) -> 32 registers, two per
-// register (column 2j in the low half).
-__device__ __forceinline__ void tmem_ld32_pack16(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.pack::16b.b32 " SAGE_REGS32 ", [%32];"
-               : SAGE_R32(r)
-               : "r"(taddr));
-}
-
 // 32 columns of FP16 values -> 16 registers, two per register.
 __device__ __forceinline__ void tmem_ld16_pack16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -248,20 +239,17 @@ __device__ __forceinline__ TcSmem<D>& tc_smem() {
 }
 
 // ------------------------------------------------------------------ kernel
-// Softmax of one tile for one row (TAIL: keys >= nvalid are masked).
-// In: S[64] int32 scores.  Out: P[16] packed E4M3 probabilities; updates
-// m and d, returns r (the factor applied to the older RO and d).
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
+
+// Float images magic + S of one row's 64 scores (exact for |S| < 2^22) and
+// the tile maximum fl32(max(S) * c); TAIL masks keys >= nvalid.
 template <bool TAIL>
-__device__ __forceinline__ float softmax_tile(const uint32_t (&S)[64], float cs, int nvalid, float& m,
-                                              float& d, uint32_t (&P)[16]) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
-  float fb[64];
+__device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int nvalid, float (&fb)[64]) {
 #pragma unroll
   for (int j = 0; j < 64; ++j) {
     fb[j] = __int_as_float((int32_t)S[j] + 0x4B400000);
     if (TAIL && j >= nvalid) fb[j] = -INFINITY;
   }
-  // tile max over the exact float images of the scores (3-input max)
   float mx[22];
 #pragma unroll
   for (int j = 0; j < 21; ++j) mx[j] = fmaxf(fmaxf(fb[3 * j], fb[3 * j + 1]), fb[3 * j + 2]);
@@ -271,36 +259,48 @@ __device__ __forceinline__ float softmax_tile(const uint32_t (&S)[64], float cs,
   const float fmx = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[21])));
   // max of fl32(S*c) = fl32(max(S)*c) since rounding is monotone and c >= 0
-  const float tmax = __fmul_rn(__fsub_rn(fmx, kMagic), cs);
-  const float m_new = fmaxf(m, tmax);
-  const float r = (m_new == m) ? 1.0f : ex2(__fsub_rn(m, m_new));
-  m = m_new;
+  return __fmul_rn(__fsub_rn(fmx, kMagic), cs);
+}
+
+// Probabilities of one row's tile against the running max m_new: the FP32
+// values p = 2^(s - m_new) go to the returned row sum, their E4M3 bytes to
+// P (key order from the low byte).
+template <bool TAIL>
+__device__ __forceinline__ float tile_exp(const float (&fb)[64], float cs, float m_new, int nvalid,
+                                          uint32_t (&P)[16]) {
   // exponent argument s - m_new as one FMA on the float image:
   // fb*c - (magic*c + m_new), with magic*c + m_new rounded once
-  const float kofs = __fmaf_rn(kMagic, cs, m_new);
-  float rs[2] = {0.0f, 0.0f};
+  const float nkofs = -__fmaf_rn(kMagic, cs, m_new);
+  float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums, two packed pairs
 #pragma unroll
   for (int q = 0; q < 16; ++q) {
     float pv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < 4; e += 2) {
       const int j = 4 * q + e;
-      pv[e] = ex2(__fmaf_rn(fb[j], cs, -kofs));
+      asm("{.reg .b64 x, c, o; mov.b64 x, {%2, %3}; mov.b64 c, {%4, %4}; mov.b64 o, {%5, %5};"
+          " fma.rn.f32x2 x, x, c, o; mov.b64 {%0, %1}, x;}"
+          : "=f"(pv[e]), "=f"(pv[e + 1])
+          : "f"(fb[j]), "f"(fb[j + 1]), "f"(cs), "f"(nkofs));
+      pv[e] = ex2(pv[e]);
+      pv[e + 1] = ex2(pv[e + 1]);
       if (TAIL && j >= nvalid) pv[e] = 0.0f;
+      if (TAIL && j + 1 >= nvalid) pv[e + 1] = 0.0f;
     }
-    // two independent packed FP32 sums (pairs of lanes of an f32x2 add)
     asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
         " mov.b64 {%0, %1}, a;}"
         : "+f"(rs[0]), "+f"(rs[1])
         : "f"(pv[0]), "f"(pv[1]));
     asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
         " mov.b64 {%0, %1}, a;}"
-        : "+f"(rs[0]), "+f"(rs[1])
+        : "+f"(rs[2]), "+f"(rs[3])
         : "f"(pv[2]), "f"(pv[3]));
-    P[q] = (uint32_t)e4m3x2(pv[0], pv[1]) | ((uint32_t)e4m3x2(pv[2], pv[3]) << 16);
+    asm("{.reg .b16 lo, hi; cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1; cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;"
+        " mov.b32 %0, {lo, hi};}"
+        : "=r"(P[q])
+        : "f"(pv[0]), "f"(pv[1]), "f"(pv[2]), "f"(pv[3]));
   }
-  d = __fadd_rn(__fmul_rn(d, r), __fadd_rn(rs[0], rs[1]));
-  return r;
+  return __fadd_rn(__fadd_rn(rs[0], rs[1]), __fadd_rn(rs[2], rs[3]));
 }
 
 template <int D>
@@ -312,85 +312,114 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int bh = b * p.H + h;
-  const int T = p.T64;
+  const int T = p.T64;            // 64-key tiles
+  const int G = (T + 1) >> 1;     // 128-key groups
   volatile int* abort_flag = &sm.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 2);  // released by both MMA issuers
+      mbar_init(&sm.kv_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.s_full[i], 1);
       mbar_init(&sm.s_free[i], 1);
       mbar_init(&sm.p_full[i], kQTile);
-      mbar_init(&sm.r_free[i], 2 * kQTile);
-    }
-    for (int i = 0; i < kOBufs; ++i) {
+      mbar_init(&sm.r_free[i], 2 * kQTile + 1);  // output owners and the PV issuer
       mbar_init(&sm.o_full[i], 1);
       mbar_init(&sm.o_free[i], 2 * kQTile);
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.m_full[q][i], 32);
     }
+    mbar_init(&sm.fin, 2 * kQTile);
     mbar_init(&sm.done, kQTile);
-    mbar_init(&sm.drain, 1);
-    mbar_init(&sm.drain2, 1);
+    mbar_init(&sm.drain_qk, 1);
+    mbar_init(&sm.drain_pv, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (warp == kQkWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp < 4) {
+  if (warp < 8) {
     // ------------------------------------------------ QK / softmax owners
-    const int i = threadIdx.x;  // row within the tile = TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int quad = warp & 3, par = warp >> 2;  // rows 32*quad.., tiles t % 2 == par
+    const int i = quad * 32 + lane;              // row within the tile = TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int row = qt * kQTile + i;
     const int grp = row / kQGroup;
     const float qs = grp < p.G32 ? p.q_scale[(size_t)bh * p.G32 + grp] : 0.0f;
     const float* ksc = p.k_scale + (size_t)bh * T;
     const int ntail = p.N - (T - 1) * kKTile;  // valid keys of the last tile
-    float m = -INFINITY, d = 0.0f;
-    float ks_next = ksc[0];
-    for (int t = 0; t < T; ++t) {
-      const int bi = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      const float ks = ks_next;
-      if (t + 1 < T) ks_next = ksc[t + 1];
-      if (!wait_bounded(&sm.s_full[bi], ph, abort_flag, p.status, 1, p.wait_limit)) break;
+    float m_own = -INFINITY, d_own = 0.0f;     // this warp's latest running max and partial denominator
+    for (int t = par; t < T; t += 2) {
+      const int g = t >> 1, sb = g & 1;
+      const uint32_t cols = kColS + 128 * sb + 64 * par;
+      const float ks = ksc[t];
+      if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) break;
       tc_fence_after();
       uint32_t S[64];
-      tmem_ld64(lane_addr + kColS + 64 * bi, S);
+      tmem_ld64(lane_addr + cols, S);
       tmem_wait_ld();
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
+      const bool tail = t + 1 == T && ntail != kKTile;
+      float fb[64];
+      const float tmax = tail ? tile_max<true>(S, cs, ntail, fb) : tile_max<false>(S, cs, kKTile, fb);
+      // running max: m(t) = max(m(t-1), tile max), m(t-1) from the partner warp
+      float m_prev = -INFINITY;
+      if (t > 0) {
+        if (!wait_bounded(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1), abort_flag, p.status, 15,
+                          p.wait_limit))
+          break;
+        m_prev = sm.m_x[par ^ 1][i];
+      }
+      const float m_new = fmaxf(m_prev, tmax);
+      sm.m_x[par][i] = m_new;
+      mbar_arrive(&sm.m_full[quad][par]);
+      const float r = (m_new == m_prev) ? 1.0f : ex2(__fsub_rn(m_prev, m_new));
       uint32_t P[16];
-      float r;
-      if (t + 1 < T || ntail == kKTile) r = softmax_tile<false>(S, cs, kKTile, m, d, P);
-      else r = softmax_tile<true>(S, cs, ntail, m, d, P);
-      tmem_st16(lane_addr + kColS + 64 * bi, P);  // E4M3 P over the first 16 score columns
+      const float rs = tail ? tile_exp<true>(fb, cs, m_new, ntail, P) : tile_exp<false>(fb, cs, m_new, kKTile, P);
+      // this warp's partial denominator, carried from its previous tile's max
+      d_own = (m_own == m_new) ? __fadd_rn(d_own, rs) : __fadd_rn(__fmul_rn(d_own, ex2(__fsub_rn(m_own, m_new))), rs);
+      m_own = m_new;
+      tmem_st16(lane_addr + cols, P);  // E4M3 P over the first 16 score columns of the tile
       tmem_wait_st();
-      if (!wait_bounded(&sm.r_free[bi], ph ^ 1u, abort_flag, p.status, 2, p.wait_limit)) break;
-      sm.r_ring[bi][i] = r;
+      if (!wait_bounded(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 2, p.wait_limit))
+        break;
+      sm.r_ring[par][i] = r;
       tc_fence_before();
-      mbar_arrive(&sm.p_full[bi]);
+      mbar_arrive(&sm.p_full[par]);
     }
-    sm.rcp[i] = __frcp_rn(d);
-    mbar_arrive(&sm.done);
-  } else if (warp < 12) {
+    // merge the two partial denominators at the final running max
+    sm.m_fin[par][i] = m_own;
+    sm.d_fin[par][i] = d_own;
+    mbar_arrive(&sm.fin);
+    if (par == 0) {
+      if (wait_bounded(&sm.fin, 0, abort_flag, p.status, 16, p.wait_limit)) {
+        const float m0 = sm.m_fin[0][i], m1 = sm.m_fin[1][i];
+        const float mf = fmaxf(m0, m1);
+        const float d0 = m0 == mf ? sm.d_fin[0][i] : __fmul_rn(sm.d_fin[0][i], ex2(__fsub_rn(m0, mf)));
+        const float d1 = m1 == mf ? sm.d_fin[1][i] : __fmul_rn(sm.d_fin[1][i], ex2(__fsub_rn(m1, mf)));
+        sm.rcp[i] = __frcp_rn(__fadd_rn(d0, d1));
+      }
+      mbar_arrive(&sm.done);
+    }
+  } else if (warp < 16) {
     // ---------------------------------------- output owners (half rows)
-    const int i = (warp & 3) * 32 + lane;      // row within the tile
-    const int c_base = warp < 8 ? 0 : DH;      // this thread's output columns
-    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const int quad = warp & 3;
+    const int i = quad * 32 + lane;            // row within the tile
+    const int c_base = warp < 12 ? 0 : DH;     // this thread's output columns
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     float RO[DH];
 #pragma unroll
     for (int c = 0; c < DH; ++c) RO[c] = 0.0f;
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
-      if (!wait_bounded(&sm.p_full[bi], ph, abort_flag, p.status, 3, p.wait_limit)) break;
+      if (!wait_bounded(&sm.p_full[bi], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 3, p.wait_limit)) break;
       const float r = sm.r_ring[bi][i];
       mbar_arrive(&sm.r_free[bi]);
       if (r != 1.0f) {
@@ -403,31 +432,31 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
 #pragma unroll
-      for (int sl = 0; sl < 2; ++sl) {
-        const int k = 2 * t + sl, ob = k % kOBufs;  // position in the buffer ring
-        if (!wait_bounded(&sm.o_full[ob], (uint32_t)((k / kOBufs) & 1), abort_flag, p.status, 4, p.wait_limit)) {
+      for (int sl = 0; sl < 2; ++sl) {  // K32 slice sl of tile t sits in buffer sl
+        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        uint32_t hv[DH / 2];
-        if (DH == 64) {
-          tmem_ld32_pack16(lane_addr + kColO + 128 * ob + c_base, *reinterpret_cast<uint32_t(*)[32]>(hv));
-        } else {
-          tmem_ld16_pack16(lane_addr + kColO + 128 * ob + c_base, *reinterpret_cast<uint32_t(*)[16]>(hv));
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&sm.o_free[ob]);  // the buffer may be overwritten now
-        // RO += float(tmp), one rounding per element (float(tmp) is exact):
-        // widen the FP16 pair, then one packed FP32x2 add
+        // 32 columns at a time (16 registers of FP16 pairs); the buffer is
+        // released once the last columns are in registers
 #pragma unroll
-        for (int j = 0; j < DH / 2; ++j) {
-          asm("{.reg .b16 lo, hi; .reg .f32 a, b; .reg .b64 x, y;"
-              " mov.b32 {lo, hi}, %2; cvt.f32.f16 a, lo; cvt.f32.f16 b, hi;"
-              " mov.b64 x, {a, b}; mov.b64 y, {%0, %1}; add.rn.f32x2 y, y, x; mov.b64 {%0, %1}, y;}"
-              : "+f"(RO[2 * j]), "+f"(RO[2 * j + 1])
-              : "r"(hv[j]));
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          uint32_t hv[16];
+          tmem_ld16_pack16(lane_addr + kColO + 128 * sl + c_base + c0, hv);
+          tmem_wait_ld();
+          if (c0 + 32 >= DH) {
+            tc_fence_before();
+            mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
+          }
+          // RO += float(tmp), one rounding per element (float(tmp) is exact):
+          // one mixed-precision add (FP16 operand, FP32 accumulator) each
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            asm("{.reg .b16 lo, hi; mov.b32 {lo, hi}, %2; add.rn.f32.f16 %0, lo, %0; add.rn.f32.f16 %1, hi, %1;}"
+                : "+f"(RO[c0 + 2 * j]), "+f"(RO[c0 + 2 * j + 1])
+                : "r"(hv[j]));
+          }
         }
       }
     }
@@ -456,82 +485,83 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       int issued = 0;
       mbar_expect_tx(&sm.q_full, kQTile * D);
       tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
-      for (int t = 0; t < T; ++t) {
-        const int st = t % kStages;
-        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((t / kStages) & 1) ^ 1), abort_flag, p.status, 6,
+      for (int g = 0; g < G; ++g) {
+        const int st = g % kStages;
+        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((g / kStages) & 1) ^ 1), abort_flag, p.status, 6,
                           p.wait_limit))
           break;
-        if (t == p.stall_tile) continue;  // test hook: this tile never arrives
-        mbar_expect_tx(&sm.kv_full[st], 2 * kKTile * D);
-        tma_load_3d(sm.k[st], &tm_k, 0, t * kKTile, bh, &sm.kv_full[st]);
-        tma_load_3d(sm.v[st], &tm_v, t * kKTile, 0, bh, &sm.kv_full[st]);
-        issued = t + 1;
+        if (p.stall_tile >= 0 && p.stall_tile / 2 == g) continue;  // test hook: this stage never arrives
+        mbar_expect_tx(&sm.kv_full[st], 2 * kGroup * D);
+        tma_load_3d(sm.k[st], &tm_k, 0, g * kGroup, bh, &sm.kv_full[st]);
+        tma_load_3d(sm.v[st], &tm_v, g * kGroup, 0, bh, &sm.kv_full[st]);
+        issued = g + 1;
       }
       // leave no copy in flight: wait for every issued stage and for Q
       wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
       for (int u = max(0, issued - kStages); u < issued; ++u)
-        if (u != p.stall_tile)
+        if (!(p.stall_tile >= 0 && p.stall_tile / 2 == u))
           wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8,
                        p.wait_limit, false);
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------- QK issuer
+  } else if (warp == kQkWarp) {
+    // ----------------------------------------------------------- QK issuer
     if (lane == 0) {
-      const uint32_t iqk = idesc_qk();
+      const uint32_t iqk = idesc_qk(kGroup);
       const uint64_t qdesc = smem_desc(sm.q, D);
       bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
-      for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kStages, bi = t & 1;
-        if (!wait_bounded(&sm.kv_full[st], (uint32_t)((t / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
-          break;
-        // PV(t-2) read its probabilities from this score buffer
-        if (!wait_bounded(&sm.s_free[bi], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit))
+      for (int g = 0; ok && g < G; ++g) {
+        const int st = g % kStages, sb = g & 1;
+        // the buffer's last probabilities (group g - 2) have been read by PV
+        if (!wait_bounded(&sm.s_free[sb], (uint32_t)(((g >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit) ||
+            !wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
           break;
         tc_fence_after();
         const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8_ss(tmem + kColS + 64 * bi, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
-        tc_commit(&sm.s_full[bi]);
-        tc_commit(&sm.kv_empty[st]);
+          mma_i8_ss(tmem + kColS + 128 * sb, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
+        tc_commit(&sm.s_full[sb]);
       }
       // no MMA may still be writing TMEM when it is freed
-      tc_commit(&sm.drain);
-      wait_bounded(&sm.drain, 0, abort_flag, nullptr, 14, p.wait_limit, false);
+      tc_commit(&sm.drain_qk);
+      wait_bounded(&sm.drain_qk, 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
     __syncwarp();
   } else if (warp == kPvWarp) {
-    // ------------------------------------------------------- PV issuer
+    // ----------------------------------------------------------- PV issuer
     if (lane == 0) {
       const uint32_t ipv = idesc_pv<D>();
-      bool ok = true;
-      for (int u = 0; ok && u < T; ++u) {
-        const int bu = u & 1, su = u % kStages;
-        // PV(u): two K32 slices, each into its own FP16 buffer from zero
-        if (!wait_bounded(&sm.p_full[bu], (uint32_t)((u >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
-        // V(u) arrived with K(u) (already waited on by the QK issuer)
-        if (!wait_bounded(&sm.kv_full[su], (uint32_t)((u / kStages) & 1), abort_flag, p.status, 16, p.wait_limit))
+      for (int t = 0; t < T; ++t) {
+        const int g = t >> 1, sb = g & 1, st = g % kStages, half = t & 1;
+        if (!wait_bounded(&sm.p_full[half], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
+        // seen: the softmax owners may complete this p_full slot again (tile t + 2)
+        mbar_arrive(&sm.r_free[half]);
+        // the V^T stage arrived with the K stage the QK issuer waited for
+        if (half == 0 &&
+            !wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 18, p.wait_limit))
           break;
         tc_fence_after();
-        const uint64_t vdesc = smem_desc(sm.v[su], kKTile);
+        // this tile's 64 keys within the stage's 128-byte V^T rows
+        const uint64_t vdesc = smem_desc(sm.v[st], kGroup) + 4 * half;
+        bool ok = true;
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
-          const int k = 2 * u + sl, ob = k % kOBufs;
-          if (!wait_bounded(&sm.o_free[ob], (uint32_t)(((k / kOBufs) & 1) ^ 1), abort_flag, p.status, 13,
-                            p.wait_limit)) {
+          if (!wait_bounded(&sm.o_free[sl], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_f8_ts(tmem + kColO + 128 * ob, tmem + kColS + 64 * bu + 8 * sl, vdesc + 2 * sl, ipv, 0);
-          tc_commit(&sm.o_full[ob]);
+          mma_f8_ts(tmem + kColO + 128 * sl, tmem + kColS + 128 * sb + 64 * half + 8 * sl, vdesc + 2 * sl, ipv, 0);
+          tc_commit(&sm.o_full[sl]);
         }
         if (!ok) break;
-        tc_commit(&sm.s_free[bu]);
-        tc_commit(&sm.kv_empty[su]);
+        if (half == 1 || t + 1 == T) {  // the group's probabilities and K/V stage are consumed
+          tc_commit(&sm.s_free[sb]);
+          tc_commit(&sm.kv_empty[st]);
+        }
       }
-      tc_commit(&sm.drain2);
-      wait_bounded(&sm.drain2, 0, abort_flag, nullptr, 15, p.wait_limit, false);
+      tc_commit(&sm.drain_pv);
+      wait_bounded(&sm.drain_pv, 0, abort_flag, nullptr, 17, p.wait_limit, false);
     }
     __syncwarp();
   }
@@ -539,7 +569,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_free(tmem, kTmemCols);
+  if (warp == kQkWarp) tmem_free(tmem, kTmemCols);
 }
 
 // ------------------------------------------------ debug: one score tile
@@ -558,7 +588,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (warp == kQkWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -566,11 +596,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (warp == kLoadWarp && lane == 0) {
     mbar_expect_tx(&sm.q_full, kQTile * D);
     tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
-    mbar_expect_tx(&sm.kv_full[0], kKTile * D);
+    mbar_expect_tx(&sm.kv_full[0], kGroup * D);  // a full stage box; its first 64 keys are the tile
     tma_load_3d(sm.k[0], &tm_k, 0, kt * kKTile, bh, &sm.kv_full[0]);
     wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
     wait_bounded(&sm.kv_full[0], 0, abort_flag, nullptr, 8, p.wait_limit, false);
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kQkWarp) {
     if (lane == 0) {
       bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit) &&
                 wait_bounded(&sm.kv_full[0], 0, abort_flag, p.status, 10, p.wait_limit);
@@ -579,7 +609,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const uint64_t qdesc = smem_desc(sm.q, D), kdesc = smem_desc(sm.k[0], D);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8_ss(tmem + kColS, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk(), kk > 0);
+          mma_i8_ss(tmem + kColS, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk(kKTile), kk > 0);
       }
       tc_commit(&sm.s_full[0]);
       wait_bounded(&sm.s_full[0], 0, abort_flag, nullptr, 14, p.wait_limit, false);
@@ -598,7 +628,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == kMmaWarp) tmem_free(tmem, kTmemCols);
+  if (warp == kQkWarp) tmem_free(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------- host
@@ -650,8 +680,8 @@ int launch_tc(const AttnParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const uint64_t bh = (uint64_t)p.B * p.H;
   if (!make_map(&mq, p.q8, D, p.Nq, bh, D, (uint64_t)p.Nq * D, D, kQTile) ||
-      !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kKTile) ||
-      !make_map(&mv, p.v8, p.Nk, D, bh, p.Nk, (uint64_t)D * p.Nk, kKTile, D))
+      !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kGroup) ||
+      !make_map(&mv, p.v8, p.Nk, D, bh, p.Nk, (uint64_t)D * p.Nk, kGroup, D))
     return SAGE_ERR_CUDA;
   auto* fn = attn_tc_kernel<D>;
   const size_t smem = smem_bytes<D>();
@@ -666,7 +696,7 @@ int launch_dbg_tc(const AttnParams& p, int b, int h, int qt, int kt, int32_t* s_
   CUtensorMap mq, mk;
   const uint64_t bh = (uint64_t)p.B * p.H;
   if (!make_map(&mq, p.q8, D, p.Nq, bh, D, (uint64_t)p.Nq * D, D, kQTile) ||
-      !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kKTile))
+      !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kGroup))
     return SAGE_ERR_CUDA;
   auto* fn = debug_qk_tc_kernel<D>;
   const size_t smem = smem_bytes<D>();

@@ -47,6 +47,8 @@ namespace sage {
 namespace {
 
 constexpr int kThreadsTC = 608;
+constexpr int kSoftWarp0 = 0;  // warps 0-7: softmax owners
+constexpr int kOutWarp0 = 8;   // warps 8-15: output owners
 constexpr int kLoadWarp = 16;
 constexpr int kQkWarp = 17;    // QK issuer; also allocates and frees the tensor memory
 constexpr int kPvWarp = 18;    // PV issuer
@@ -215,6 +217,25 @@ __device__ __forceinline__ void tmem_ld16_pack16(uint32_t taddr, uint32_t (&r)[1
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 columns of 32 bits -> 16 registers.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// Wait for this thread's TMEM loads; the registers pass through the wait so
+// that no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -241,51 +262,49 @@ __device__ __forceinline__ TcSmem<D>& tc_smem() {
 // ------------------------------------------------------------------ kernel
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
 
-// Float images magic + S of one row's 64 scores (exact for |S| < 2^22) and
-// the tile maximum fl32(max(S) * c); TAIL masks keys >= nvalid.
+// Tile maximum fl32(max(S) * c) of one row's 64 scores (the max of the
+// integers is exact, and rounding is monotone with c >= 0); TAIL masks keys
+// >= nvalid.
 template <bool TAIL>
-__device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int nvalid, float (&fb)[64]) {
+__device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int nvalid) {
+  int mx[32];
 #pragma unroll
-  for (int j = 0; j < 64; ++j) {
-    fb[j] = __int_as_float((int32_t)S[j] + 0x4B400000);
-    if (TAIL && j >= nvalid) fb[j] = -INFINITY;
+  for (int j = 0; j < 32; ++j) {
+    const int a = (TAIL && 2 * j >= nvalid) ? INT_MIN : (int)S[2 * j];
+    const int b = (TAIL && 2 * j + 1 >= nvalid) ? INT_MIN : (int)S[2 * j + 1];
+    mx[j] = max(a, b);
   }
-  float mx[22];
 #pragma unroll
-  for (int j = 0; j < 21; ++j) mx[j] = fmaxf(fmaxf(fb[3 * j], fb[3 * j + 1]), fb[3 * j + 2]);
-  mx[21] = fb[63];
+  for (int w = 16; w > 0; w >>= 1)
 #pragma unroll
-  for (int j = 0; j < 7; ++j) mx[j] = fmaxf(fmaxf(mx[3 * j], mx[3 * j + 1]), mx[3 * j + 2]);
-  const float fmx = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[21])));
-  // max of fl32(S*c) = fl32(max(S)*c) since rounding is monotone and c >= 0
-  return __fmul_rn(__fsub_rn(fmx, kMagic), cs);
+    for (int j = 0; j < w; ++j) mx[j] = max(mx[j], mx[j + w]);
+  return __fmul_rn(__int2float_rn(mx[0]), cs);
 }
 
-// Probabilities of one row's tile against the running max m_new: the FP32
-// values p = 2^(s - m_new) go to the returned row sum, their E4M3 bytes to
-// P (key order from the low byte).
+// Probabilities of 16 of a row's keys (k0..k0+15) against the running max:
+// p = 2^(s - m_new) in FP32 into the partial sums rs, E4M3 bytes (key order
+// from the low byte) into P[k0/4 ..].  nkofs = -(magic*c + m_new), rounded once.
 template <bool TAIL>
-__device__ __forceinline__ float tile_exp(const float (&fb)[64], float cs, float m_new, int nvalid,
-                                          uint32_t (&P)[16]) {
-  // exponent argument s - m_new as one FMA on the float image:
-  // fb*c - (magic*c + m_new), with magic*c + m_new rounded once
-  const float nkofs = -__fmaf_rn(kMagic, cs, m_new);
-  float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums, two packed pairs
+__device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, float cs, float nkofs, int nvalid,
+                                          float (&rs)[4], uint32_t (&P)[16]) {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
+  for (int q = 0; q < 4; ++q) {
     float pv[4];
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
       const int j = 4 * q + e;
+      // exponent arguments fl32(fb*c - kofs) on the exact float images
+      // fb = magic + S, two per packed FMA
+      const float f0 = __int_as_float((int32_t)Sc[j] + 0x4B400000);
+      const float f1 = __int_as_float((int32_t)Sc[j + 1] + 0x4B400000);
       asm("{.reg .b64 x, c, o; mov.b64 x, {%2, %3}; mov.b64 c, {%4, %4}; mov.b64 o, {%5, %5};"
           " fma.rn.f32x2 x, x, c, o; mov.b64 {%0, %1}, x;}"
           : "=f"(pv[e]), "=f"(pv[e + 1])
-          : "f"(fb[j]), "f"(fb[j + 1]), "f"(cs), "f"(nkofs));
+          : "f"(f0), "f"(f1), "f"(cs), "f"(nkofs));
       pv[e] = ex2(pv[e]);
       pv[e + 1] = ex2(pv[e + 1]);
-      if (TAIL && j >= nvalid) pv[e] = 0.0f;
-      if (TAIL && j + 1 >= nvalid) pv[e + 1] = 0.0f;
+      if (TAIL && k0 + j >= nvalid) pv[e] = 0.0f;
+      if (TAIL && k0 + j + 1 >= nvalid) pv[e + 1] = 0.0f;
     }
     asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
         " mov.b64 {%0, %1}, a;}"
@@ -297,9 +316,32 @@ __device__ __forceinline__ float tile_exp(const float (&fb)[64], float cs, float
         : "f"(pv[2]), "f"(pv[3]));
     asm("{.reg .b16 lo, hi; cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1; cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;"
         " mov.b32 %0, {lo, hi};}"
-        : "=r"(P[q])
+        : "=r"(P[k0 / 4 + q])
         : "f"(pv[0]), "f"(pv[1]), "f"(pv[2]), "f"(pv[3]));
   }
+}
+
+// The exponential pass over a tile: the scores are read again from TMEM in
+// four 16-column chunks (double-buffered), so that the registers of the max
+// pass are free.  Returns the FP32 row sum.
+template <bool TAIL>
+__device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new, int nvalid, uint32_t (&P)[16]) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
+  const float nkofs = -__fmaf_rn(kMagic, cs, m_new);
+  float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  uint32_t A[16], Bc[16];
+  tmem_ld16(taddr, A);
+  tmem_wait_ld16(A);
+  tmem_ld16(taddr + 16, Bc);
+  chunk_exp<TAIL>(A, 0, cs, nkofs, nvalid, rs, P);
+  tmem_wait_ld16(Bc);
+  tmem_ld16(taddr + 32, A);
+  chunk_exp<TAIL>(Bc, 16, cs, nkofs, nvalid, rs, P);
+  tmem_wait_ld16(A);
+  tmem_ld16(taddr + 48, Bc);
+  chunk_exp<TAIL>(A, 32, cs, nkofs, nvalid, rs, P);
+  tmem_wait_ld16(Bc);
+  chunk_exp<TAIL>(Bc, 48, cs, nkofs, nvalid, rs, P);
   return __fadd_rn(__fadd_rn(rs[0], rs[1]), __fadd_rn(rs[2], rs[3]));
 }
 
@@ -344,9 +386,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp < 8) {
+  if (warp >= kSoftWarp0 && warp < kOutWarp0) {
     // ------------------------------------------------ QK / softmax owners
-    const int quad = warp & 3, par = warp >> 2;  // rows 32*quad.., tiles t % 2 == par
+    const int quad = warp & 3, par = (warp - kSoftWarp0) >> 2;  // rows 32*quad.., tiles t % 2 == par
     const int i = quad * 32 + lane;              // row within the tile = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const int row = qt * kQTile + i;
@@ -355,10 +397,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const float* ksc = p.k_scale + (size_t)bh * T;
     const int ntail = p.N - (T - 1) * kKTile;  // valid keys of the last tile
     float m_own = -INFINITY, d_own = 0.0f;     // this warp's latest running max and partial denominator
+    float ks_next = par < T ? ksc[par] : 0.0f;  // K scale of this warp's next tile, loaded a tile ahead
     for (int t = par; t < T; t += 2) {
       const int g = t >> 1, sb = g & 1;
       const uint32_t cols = kColS + 128 * sb + 64 * par;
-      const float ks = ksc[t];
+      const float ks = ks_next;
+      if (t + 2 < T) ks_next = ksc[t + 2];
       if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) break;
       tc_fence_after();
       uint32_t S[64];
@@ -366,8 +410,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tmem_wait_ld();
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
       const bool tail = t + 1 == T && ntail != kKTile;
-      float fb[64];
-      const float tmax = tail ? tile_max<true>(S, cs, ntail, fb) : tile_max<false>(S, cs, kKTile, fb);
+      const float tmax = tail ? tile_max<true>(S, cs, ntail) : tile_max<false>(S, cs, kKTile);
       // running max: m(t) = max(m(t-1), tile max), m(t-1) from the partner warp
       float m_prev = -INFINITY;
       if (t > 0) {
@@ -381,7 +424,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_arrive(&sm.m_full[quad][par]);
       const float r = (m_new == m_prev) ? 1.0f : ex2(__fsub_rn(m_prev, m_new));
       uint32_t P[16];
-      const float rs = tail ? tile_exp<true>(fb, cs, m_new, ntail, P) : tile_exp<false>(fb, cs, m_new, kKTile, P);
+      const float rs = tail ? tile_exp<true>(lane_addr + cols, cs, m_new, ntail, P)
+                            : tile_exp<false>(lane_addr + cols, cs, m_new, kKTile, P);
       // this warp's partial denominator, carried from its previous tile's max
       d_own = (m_own == m_new) ? __fadd_rn(d_own, rs) : __fadd_rn(__fmul_rn(d_own, ex2(__fsub_rn(m_own, m_new))), rs);
       m_own = m_new;
@@ -407,11 +451,11 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
       mbar_arrive(&sm.done);
     }
-  } else if (warp < 16) {
+  } else if (warp < kLoadWarp) {
     // ---------------------------------------- output owners (half rows)
     const int quad = warp & 3;
-    const int i = quad * 32 + lane;            // row within the tile
-    const int c_base = warp < 12 ? 0 : DH;     // this thread's output columns
+    const int i = quad * 32 + lane;                  // row within the tile
+    const int c_base = warp < kOutWarp0 + 4 ? 0 : DH;  // this thread's output columns
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     float RO[DH];
 #pragma unroll
@@ -615,14 +659,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       wait_bounded(&sm.s_full[0], 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp >= kSoftWarp0 && warp < kSoftWarp0 + 4) {
     if (wait_bounded(&sm.s_full[0], 0, abort_flag, p.status, 1, p.wait_limit) && !*abort_flag) {
       tc_fence_after();
+      const int quad = warp & 3;
       uint32_t S[64];
-      tmem_ld64(tmem + ((uint32_t)(warp * 32) << 16) + kColS, S);
+      tmem_ld64(tmem + ((uint32_t)(quad * 32) << 16) + kColS, S);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 64; ++j) s_out[threadIdx.x * kKTile + j] = (int32_t)S[j];
+      for (int j = 0; j < 64; ++j) s_out[(quad * 32 + lane) * kKTile + j] = (int32_t)S[j];
     }
   }
   tc_fence_before();

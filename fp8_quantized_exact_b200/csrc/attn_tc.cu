@@ -102,10 +102,12 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
 }
 
 // Bounded wait.  Returns false if the CTA is aborting or the wait ran out
-// (then the status word and the abort flag are set).
+// (then the status word and the abort flag are set).  A phase that is
+// already complete costs one try_wait.
 __device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volatile int* abort_flag,
                                              DeviceStatus* st, int where, long long limit,
                                              bool honour_abort = true) {
+  if (mbar_try(b, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try(b, parity)) return true;

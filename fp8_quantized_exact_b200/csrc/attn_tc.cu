@@ -410,14 +410,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       uint32_t S[64];
       tmem_ld64(lane_addr + cols, S);
       tmem_wait_ld();
+      // test the handoffs of this tile early; their latency overlaps the max pass
+      const bool m_ready = t == 0 || mbar_try(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1));
+      const bool r_ready = mbar_try(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1));
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
       const bool tail = t + 1 == T && ntail != kKTile;
       const float tmax = tail ? tile_max<true>(S, cs, ntail) : tile_max<false>(S, cs, kKTile);
       // running max: m(t) = max(m(t-1), tile max), m(t-1) from the partner warp
       float m_prev = -INFINITY;
       if (t > 0) {
-        if (!wait_bounded(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1), abort_flag, p.status, 15,
-                          p.wait_limit))
+        if (!m_ready && !wait_bounded(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1), abort_flag,
+                                      p.status, 15, p.wait_limit))
           break;
         m_prev = sm.m_x[par ^ 1][i];
       }
@@ -433,7 +436,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       m_own = m_new;
       tmem_st16(lane_addr + cols, P);  // E4M3 P over the first 16 score columns of the tile
       tmem_wait_st();
-      if (!wait_bounded(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 2, p.wait_limit))
+      if (!r_ready &&
+          !wait_bounded(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 2, p.wait_limit))
         break;
       sm.r_ring[par][i] = r;
       tc_fence_before();

@@ -18,12 +18,18 @@
 //               at the end it applies 1/d and the V scale and stores BF16.
 //   warp 16     TMA producer: the Q tile once, then K and V^T stages of 128
 //               keys (two tiles) into a ring of shared-memory stages.
-//   warp 17     QK issuer (one thread): per 128-key group four INT8 MMAs
-//               (N = 128, K = 32 each) into one of two TMEM score buffers.
-//   warp 18     PV issuer (one thread): once a tile's probabilities are in,
+//   warp 17     QK issuer: per 128-key group four INT8 MMAs (N = 128, K = 32
+//               each) into one of two TMEM score buffers.
+//   warp 18     PV issuer: once a tile's probabilities are in,
 //               per K32 slice one E4M3 MMA, with the probabilities as the TMEM
 //               A operand, into an FP16 accumulator that starts at zero (the
 //               instantaneous buffer), one TMEM buffer per slice.
+// The producer and issuer warps run their loops and waits with all 32 lanes
+// (lane 0 issues the copies, MMAs, commits and arrivals), which keeps them off
+// the slow divergent path.  Each wait there is followed by __syncwarp, so lane
+// 0 acts only after every lane has seen the phase; as every next phase of
+// those barriers needs an action of lane 0, the phase stays complete while
+// any lane still polls, and all lanes reach the same outcome.
 // Handoffs are block-scope mbarriers; tcgen05.commit signals MMA completion.
 // Every wait is bounded: a wait that runs out records SAGE_ERR_TIMEOUT in
 // the status word, raises a CTA-wide abort flag, and every role then leaves
@@ -531,89 +537,100 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     }
   } else if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int issued = 0;
+    // The whole warp runs the loop and the waits; lane 0 issues the copies.
+    const bool leader = lane == 0;
+    int issued = 0;
+    if (leader) {
       mbar_expect_tx(&sm.q_full, kQTile * D);
       tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
-      for (int g = 0; g < G; ++g) {
-        const int st = g % kStages;
-        if (!wait_bounded(&sm.kv_empty[st], (uint32_t)(((g / kStages) & 1) ^ 1), abort_flag, p.status, 6,
-                          p.wait_limit))
-          break;
-        if (p.stall_tile >= 0 && p.stall_tile / 2 == g) continue;  // test hook: this stage never arrives
+    }
+    for (int g = 0; g < G; ++g) {
+      const int st = g % kStages;
+      const bool ok =
+          wait_bounded(&sm.kv_empty[st], (uint32_t)(((g / kStages) & 1) ^ 1), abort_flag, p.status, 6, p.wait_limit);
+      __syncwarp();  // every lane has seen the phase before lane 0 acts on it
+      if (!ok) break;
+      if (p.stall_tile >= 0 && p.stall_tile / 2 == g) continue;  // test hook: this stage never arrives
+      if (leader) {
         mbar_expect_tx(&sm.kv_full[st], 2 * kGroup * D);
         tma_load_3d(sm.k[st], &tm_k, 0, g * kGroup, bh, &sm.kv_full[st]);
         tma_load_3d(sm.v[st], &tm_v, g * kGroup, 0, bh, &sm.kv_full[st]);
-        issued = g + 1;
       }
-      // leave no copy in flight: wait for every issued stage and for Q
-      wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
-      for (int u = max(0, issued - kStages); u < issued; ++u)
-        if (!(p.stall_tile >= 0 && p.stall_tile / 2 == u))
-          wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8,
-                       p.wait_limit, false);
+      issued = g + 1;
     }
+    // leave no copy in flight: wait for every issued stage and for Q
+    wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
+    for (int u = max(0, issued - kStages); u < issued; ++u)
+      if (!(p.stall_tile >= 0 && p.stall_tile / 2 == u))
+        wait_bounded(&sm.kv_full[u % kStages], (uint32_t)((u / kStages) & 1), abort_flag, nullptr, 8,
+                     p.wait_limit, false);
   } else if (warp == kQkWarp) {
     // ----------------------------------------------------------- QK issuer
-    if (lane == 0) {
-      const uint32_t iqk = idesc_qk(kGroup);
-      const uint64_t qdesc = smem_desc(sm.q, D);
-      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
-      for (int g = 0; ok && g < G; ++g) {
-        const int st = g % kStages, sb = g & 1;
-        // the buffer's last probabilities (group g - 2) have been read by PV
-        if (!wait_bounded(&sm.s_free[sb], (uint32_t)(((g >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit) ||
-            !wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 10, p.wait_limit))
-          break;
-        tc_fence_after();
+    // The whole warp runs the loop and the waits; lane 0 issues and commits.
+    const bool leader = lane == 0;
+    const uint32_t iqk = idesc_qk(kGroup);
+    const uint64_t qdesc = smem_desc(sm.q, D);
+    bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit);
+    __syncwarp();
+    for (int g = 0; ok && g < G; ++g) {
+      const int st = g % kStages, sb = g & 1;
+      // the buffer's last probabilities (group g - 2) have been read by PV
+      ok = wait_bounded(&sm.s_free[sb], (uint32_t)(((g >> 1) & 1) ^ 1), abort_flag, p.status, 11, p.wait_limit) &&
+           wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 10, p.wait_limit);
+      __syncwarp();  // every lane has seen the phases before lane 0 acts on them
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
         const uint64_t kdesc = smem_desc(sm.k[st], D);
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk)
           mma_i8_ss(tmem + kColS + 128 * sb, qdesc + 2 * kk, kdesc + 2 * kk, iqk, kk > 0);
         tc_commit(&sm.s_full[sb]);
       }
-      // no MMA may still be writing TMEM when it is freed
-      tc_commit(&sm.drain_qk);
-      wait_bounded(&sm.drain_qk, 0, abort_flag, nullptr, 14, p.wait_limit, false);
     }
+    // no MMA may still be writing TMEM when it is freed
     __syncwarp();
+    if (leader) tc_commit(&sm.drain_qk);
+    __syncwarp();
+    wait_bounded(&sm.drain_qk, 0, abort_flag, nullptr, 14, p.wait_limit, false);
   } else if (warp == kPvWarp) {
     // ----------------------------------------------------------- PV issuer
-    if (lane == 0) {
-      const uint32_t ipv = idesc_pv<D>();
-      for (int t = 0; t < T; ++t) {
-        const int g = t >> 1, sb = g & 1, st = g % kStages, half = t & 1;
-        if (!wait_bounded(&sm.p_full[half], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 12, p.wait_limit)) break;
+    // The whole warp runs the loop and the waits; lane 0 issues, commits and arrives.
+    const bool leader = lane == 0;
+    const uint32_t ipv = idesc_pv<D>();
+    for (int t = 0; t < T; ++t) {
+      const int g = t >> 1, sb = g & 1, st = g % kStages, half = t & 1;
+      // this tile's probabilities; the V^T stage, which arrived with the K stage
+      // the QK issuer waited for; both FP16 buffers read by the output owners
+      const bool ok =
+          wait_bounded(&sm.p_full[half], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 12, p.wait_limit) &&
+          (half == 1 ||
+           wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 18, p.wait_limit)) &&
+          wait_bounded(&sm.o_free[0], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit) &&
+          wait_bounded(&sm.o_free[1], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit);
+      __syncwarp();  // every lane has seen the phases before lane 0 acts on them
+      if (!ok) break;
+      tc_fence_after();
+      if (leader) {
         // seen: the softmax owners may complete this p_full slot again (tile t + 2)
         mbar_arrive(&sm.r_free[half]);
-        // the V^T stage arrived with the K stage the QK issuer waited for
-        if (half == 0 &&
-            !wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 18, p.wait_limit))
-          break;
-        tc_fence_after();
         // this tile's 64 keys within the stage's 128-byte V^T rows
         const uint64_t vdesc = smem_desc(sm.v[st], kGroup) + 4 * half;
-        bool ok = true;
 #pragma unroll
         for (int sl = 0; sl < 2; ++sl) {
-          if (!wait_bounded(&sm.o_free[sl], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
           mma_f8_ts(tmem + kColO + 128 * sl, tmem + kColS + 128 * sb + 64 * half + 8 * sl, vdesc + 2 * sl, ipv, 0);
           tc_commit(&sm.o_full[sl]);
         }
-        if (!ok) break;
         if (half == 1 || t + 1 == T) {  // the group's probabilities and K/V stage are consumed
           tc_commit(&sm.s_free[sb]);
           tc_commit(&sm.kv_empty[st]);
         }
       }
-      tc_commit(&sm.drain_pv);
-      wait_bounded(&sm.drain_pv, 0, abort_flag, nullptr, 17, p.wait_limit, false);
     }
     __syncwarp();
+    if (leader) tc_commit(&sm.drain_pv);
+    __syncwarp();
+    wait_bounded(&sm.drain_pv, 0, abort_flag, nullptr, 17, p.wait_limit, false);
   }
 
   tc_fence_before();

@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -49,7 +50,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
-    ap.add_argument("--cpu-sample-groups", type=int, default=6)
+    ap.add_argument("--cpu-sample-groups", type=int, default=16)
     return ap.parse_args()
 
 
@@ -154,6 +155,32 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     t = torch.tensor([float(x)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def pct(xs, q):
+    """q-th percentile (nearest rank) of a list of times."""
+    ys = sorted(xs)
+    return ys[min(len(ys) - 1, max(0, math.ceil(q / 100.0 * len(ys)) - 1))]
+
+
+SMS, SM_MHZ = 148, 1965.0      # B200 SM count and maximum SM clock
+
+
+def secondary_bounds(cfg, mainloop_ms: float):
+    """The mainloop's non-tensor floors at the maximum SM clock: the MUFU
+    (one exp2 per score at 16 per clock per SM), the FP32 pipe (about 5
+    softmax operations per score plus 2*D/64 adds of the per-K32 FP16
+    buffers, 128 lanes per clock per SM) and the L2-to-SM bytes (K8 and V8
+    of a head read once per 128-row query tile)."""
+    scores = cfg.B * cfg.H * cfg.N * cfg.N
+    exp2_floor = scores / (16 * SMS * SM_MHZ * 1e6) * 1e3
+    fp32_ops = scores * (5 + 2 * cfg.D / 64)
+    fp32_floor = fp32_ops / (128 * SMS * SM_MHZ * 1e6) * 1e3
+    qtiles = -(-cfg.N // 128)
+    l2_bytes = cfg.B * cfg.H * 2 * (-(-cfg.N // 64) * 64) * cfg.D * qtiles
+    return {"mufu_exp2": scores, "mufu_floor_ms": exp2_floor, "mufu_frac": exp2_floor / mainloop_ms,
+            "fp32_ops_est": fp32_ops, "fp32_floor_ms": fp32_floor, "fp32_frac": fp32_floor / mainloop_ms,
+            "l2_to_sm_bytes": l2_bytes, "clock_mhz": SM_MHZ}
 
 
 def whole_job_tops(ops_per_rank: float, world: int, ms_per_step: float) -> float:
@@ -274,7 +301,9 @@ def main():
     ws_m = sage.workspace(sage.SAGE_OP_ATTN_FROM_QUANT, B, N, H, D, dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev_a=None, ev_b=None):
+    def step(ev_s=None, ev_a=None, ev_b=None):
+        if ev_s is not None:
+            ev_s.record(stream)
         sage.sage_quant_qk(q, k, qt["q_i8"], qt["q_scale"], qt["k_i8"], qt["k_scale"], qt["k_mean"], ws_qk)
         sage.sage_quant_v(v, qt["v_fp8"], qt["v_scale"], ws_v)
         if ev_a is not None:
@@ -296,8 +325,7 @@ def main():
         if st != sage.SAGE_OK:
             raise RuntimeError(f"device status after warm-up: {sage.sage_strerror(st)}")
 
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local, enabled=not args.no_clocks) as clk:
         barrier()
@@ -309,7 +337,8 @@ def main():
         torch.cuda.synchronize()
         barrier()
     total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
-    ml_ms = [a.elapsed_time(b) for a, b in evs]
+    ml_ms = [a.elapsed_time(b) for _, a, b in evs]
+    step_ms = [s0.elapsed_time(b) for s0, _, b in evs]
     ms_step = total_ms / args.steps
     value = whole_job_tops(cfg.ops, world, ms_step)
     ml_avg = statistics.mean(ml_ms)
@@ -354,6 +383,9 @@ def main():
                        "l2": "inputs 1.6 GB > 126 MB L2 (no flush needed)"
                        if cfg.name == "long_fused" else "see workload"},
             "mainloop_ms": ml_avg, "mainloop_ms_min": min(ml_ms), "prepass_ms": ms_step - ml_avg,
+            "percentiles_ms": {"step_p50": pct(step_ms, 50), "step_p95": pct(step_ms, 95),
+                               "mainloop_p50": pct(ml_ms, 50), "mainloop_p95": pct(ml_ms, 95)},
+            "secondary_bounds": secondary_bounds(cfg, ml_avg),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TOPS",
                          "frac": achieved / peak,
                          "peak_source": f"{src} bf16 {bf16} TFLOP/s x {NOMINAL_I8_OVER_BF16} "

@@ -36,7 +36,7 @@ METRIC = ("sage_attn_fwd effective TOPS (4*B*H*N^2*D / step time) at N=37810, H=
 UNIT = "TOPS"
 NOMINAL_I8_OVER_BF16 = 2.0        # dense INT8/FP8 : BF16 tensor peak (4.5 : 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0     # used only when MEASURED_PEAKS.json is absent
-MAINLOOP_SOURCES = ["attn_tc.cu", "attn_mma.cu", "sage_common.cuh"]
+MAINLOOP_SOURCES = ["attn_tc.cu", "attn_mma.cu", "attn_tc_f32.cu", "tc_prims.cuh", "sage_common.cuh"]
 
 
 def parse():
@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="long_fused")
-    ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync"])
+    ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -270,9 +270,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     ml = {"default": sage.SAGE_MAINLOOP_DEFAULT, "tcgen05": sage.SAGE_MAINLOOP_TCGEN05,
-          "mma_sync": sage.SAGE_MAINLOOP_MMA_SYNC}[args.mainloop]
+          "mma_sync": sage.SAGE_MAINLOOP_MMA_SYNC, "tcgen05_f32": sage.SAGE_MAINLOOP_TCGEN05_F32}[args.mainloop]
     sage.sage_set_mainloop(ml)
-    ml_name = {1: "tcgen05", 2: "mma_sync"}[sage.sage_get_mainloop()]
+    ml_name = {1: "tcgen05", 2: "mma_sync", 3: "tcgen05_f32"}[sage.sage_get_mainloop()]
 
     B, N, H, D = cfg.B, cfg.N, cfg.H, cfg.D
     inp = synth.make_inputs(cfg, seed=rank)

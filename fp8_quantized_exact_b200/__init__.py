@@ -34,6 +34,7 @@ SAGE_OP_DEBUG_QK = 4
 SAGE_MAINLOOP_DEFAULT = 0
 SAGE_MAINLOOP_TCGEN05 = 1
 SAGE_MAINLOOP_MMA_SYNC = 2
+SAGE_MAINLOOP_TCGEN05_F32 = 3  # quality-gated fast variant, not the exact contract
 
 SAGE_STATUS_BYTES = 256
 

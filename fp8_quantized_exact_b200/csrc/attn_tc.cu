@@ -48,9 +48,12 @@
 #include <cuda.h>
 
 #include "sage_common.cuh"
+#include "tc_prims.cuh"
 
 namespace sage {
 namespace {
+
+using namespace tc;
 
 constexpr int kThreadsTC = 608;
 constexpr int kSoftWarp0 = 0;  // warps 0-7: softmax owners
@@ -86,181 +89,6 @@ struct TcSmem {
   int abort_flag;
 };
 
-// ------------------------------------------------------------- primitives
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{.reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p;}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait.  Returns false if the CTA is aborting or the wait ran out
-// (then the status word and the abort flag are set).  A phase that is
-// already complete costs one try_wait.
-__device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                             DeviceStatus* st, int where, long long limit,
-                                             bool honour_abort = true) {
-  if (mbar_try(b, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try(b, parity)) return true;
-    if ((i & 31u) == 31u) {
-      if (honour_abort && *abort_flag) return false;
-      if (clock64() - t0 > limit) break;
-    }
-  }
-  *abort_flag = 1;
-  if (st && atomicCAS(&st->code, 0, (int)SAGE_ERR_TIMEOUT) == 0) {
-    st->where = where;
-    st->block = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
-  }
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-      "%4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint64_t* b) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(b))
-               : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major tile whose rows are
-// `row_bytes` (64 or 128) long, written by TMA with the matching swizzle:
-// 8-row core groups `8 * row_bytes` apart (stride byte offset), leading
-// byte offset unused for swizzled K-major layouts, descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc(const void* tile, int row_bytes) {
-  const uint32_t a = smem_u32(tile);
-  uint64_t d = (uint64_t)((a >> 4) & 0x3FFFu);
-  d |= (uint64_t)1u << 16;                                   // LBO (16 B), ignored
-  d |= (uint64_t)(((8u * row_bytes) >> 4) & 0x3FFFu) << 32;  // SBO
-  d |= (uint64_t)1u << 46;                                   // version
-  d |= (uint64_t)(row_bytes == 128 ? 2u : 4u) << 61;         // SWIZZLE_128B / SWIZZLE_64B
-  return d;
-}
-
-// Instruction descriptors: M = 128, K-major A and B.
-// QK: INT8 x INT8 -> S32, N keys.  PV: E4M3 x E4M3 -> F16, N = D.
-__host__ __device__ constexpr uint32_t idesc_qk(int n) {
-  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
-}
-template <int D>
-__host__ __device__ constexpr uint32_t idesc_pv() {
-  return ((uint32_t)(D >> 3) << 17) | ((uint32_t)(kQTile >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{.reg .pred p; setp.ne.b32 p, %4, 0; tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;}" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// 32 lanes x 64 columns of 32 bits -> 64 registers (thread t = lane base + t).
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,"
-      "%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, "
-      "[%64];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),
-        "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),
-        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
-        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),
-        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-// 32 columns of FP16 values -> 16 registers, two per register.
-__device__ __forceinline__ void tmem_ld16_pack16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.pack::16b.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// 32 lanes x 16 columns of 32 bits -> 16 registers.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-// Wait for this thread's TMEM loads; the registers pass through the wait so
-// that no use of them can be scheduled before it.
-__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                 "+r"(r[15])
-               :
-               : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
-               "r"(cols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ void tmem_free(uint32_t base, uint32_t cols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(base), "r"(cols) : "memory");
-}
-
 template <int D>
 __device__ __forceinline__ TcSmem<D>& tc_smem() {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -268,91 +96,6 @@ __device__ __forceinline__ TcSmem<D>& tc_smem() {
 }
 
 // ------------------------------------------------------------------ kernel
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
-
-// Tile maximum fl32(max(S) * c) of one row's 64 scores (the max of the
-// integers is exact, and rounding is monotone with c >= 0); TAIL masks keys
-// >= nvalid.
-template <bool TAIL>
-__device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int nvalid) {
-  int mx[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int a = (TAIL && 2 * j >= nvalid) ? INT_MIN : (int)S[2 * j];
-    const int b = (TAIL && 2 * j + 1 >= nvalid) ? INT_MIN : (int)S[2 * j + 1];
-    mx[j] = max(a, b);
-  }
-#pragma unroll
-  for (int w = 16; w > 0; w >>= 1)
-#pragma unroll
-    for (int j = 0; j < w; ++j) mx[j] = max(mx[j], mx[j + w]);
-  return __fmul_rn(__int2float_rn(mx[0]), cs);
-}
-
-// Probabilities of 16 of a row's keys (k0..k0+15) against the running max:
-// p = 2^(s - m_new) in FP32 into the partial sums rs, E4M3 bytes (key order
-// from the low byte) into P[k0/4 ..].  nkofs = -(magic*c + m_new), rounded once.
-template <bool TAIL>
-__device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, float cs, float nkofs, int nvalid,
-                                          float (&rs)[4], uint32_t (&P)[16]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float pv[4];
-#pragma unroll
-    for (int e = 0; e < 4; e += 2) {
-      const int j = 4 * q + e;
-      // exponent arguments fl32(fb*c - kofs) on the exact float images
-      // fb = magic + S, two per packed FMA
-      const float f0 = __int_as_float((int32_t)Sc[j] + 0x4B400000);
-      const float f1 = __int_as_float((int32_t)Sc[j + 1] + 0x4B400000);
-      asm("{.reg .b64 x, c, o; mov.b64 x, {%2, %3}; mov.b64 c, {%4, %4}; mov.b64 o, {%5, %5};"
-          " fma.rn.f32x2 x, x, c, o; mov.b64 {%0, %1}, x;}"
-          : "=f"(pv[e]), "=f"(pv[e + 1])
-          : "f"(f0), "f"(f1), "f"(cs), "f"(nkofs));
-      pv[e] = ex2(pv[e]);
-      pv[e + 1] = ex2(pv[e + 1]);
-      if (TAIL && k0 + j >= nvalid) pv[e] = 0.0f;
-      if (TAIL && k0 + j + 1 >= nvalid) pv[e + 1] = 0.0f;
-    }
-    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
-        " mov.b64 {%0, %1}, a;}"
-        : "+f"(rs[0]), "+f"(rs[1])
-        : "f"(pv[0]), "f"(pv[1]));
-    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
-        " mov.b64 {%0, %1}, a;}"
-        : "+f"(rs[2]), "+f"(rs[3])
-        : "f"(pv[2]), "f"(pv[3]));
-    asm("{.reg .b16 lo, hi; cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1; cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;"
-        " mov.b32 %0, {lo, hi};}"
-        : "=r"(P[k0 / 4 + q])
-        : "f"(pv[0]), "f"(pv[1]), "f"(pv[2]), "f"(pv[3]));
-  }
-}
-
-// The exponential pass over a tile: the scores are read again from TMEM in
-// four 16-column chunks (double-buffered), so that the registers of the max
-// pass are free.  Returns the FP32 row sum.
-template <bool TAIL>
-__device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new, int nvalid, uint32_t (&P)[16]) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
-  const float nkofs = -__fmaf_rn(kMagic, cs, m_new);
-  float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  uint32_t A[16], Bc[16];
-  tmem_ld16(taddr, A);
-  tmem_wait_ld16(A);
-  tmem_ld16(taddr + 16, Bc);
-  chunk_exp<TAIL>(A, 0, cs, nkofs, nvalid, rs, P);
-  tmem_wait_ld16(Bc);
-  tmem_ld16(taddr + 32, A);
-  chunk_exp<TAIL>(Bc, 16, cs, nkofs, nvalid, rs, P);
-  tmem_wait_ld16(A);
-  tmem_ld16(taddr + 48, Bc);
-  chunk_exp<TAIL>(A, 32, cs, nkofs, nvalid, rs, P);
-  tmem_wait_ld16(Bc);
-  chunk_exp<TAIL>(Bc, 48, cs, nkofs, nvalid, rs, P);
-  return __fadd_rn(__fadd_rn(rs[0], rs[1]), __fadd_rn(rs[2], rs[3]));
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -700,41 +443,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 }
 
 // ------------------------------------------------------------------- host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                  CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-
-// 3-D uint8 tensor map: dims {inner, rows, BH} with row pitch `pitch` bytes
-// and head pitch `hpitch` bytes; box {box_inner, box_rows, 1}.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t bh, uint64_t pitch,
-              uint64_t hpitch, uint32_t box_inner, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {inner, rows, bh};
-  const cuuint64_t strides[2] = {pitch, hpitch};
-  const cuuint32_t box[3] = {box_inner, box_rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUtensorMapSwizzle sw = box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 size_t smem_bytes() {
   // at least 120 KB so that a second CTA (and its 512-column TMEM request)

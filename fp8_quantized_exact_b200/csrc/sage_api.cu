@@ -120,6 +120,7 @@ int resolved_mainloop() {
     if (e && g_mainloop == SAGE_MAINLOOP_DEFAULT) {
       if (!strcmp(e, "tcgen05")) g_mainloop = SAGE_MAINLOOP_TCGEN05;
       else if (!strcmp(e, "mma_sync") || !strcmp(e, "mmasync")) g_mainloop = SAGE_MAINLOOP_MMA_SYNC;
+      else if (!strcmp(e, "tcgen05_f32")) g_mainloop = SAGE_MAINLOOP_TCGEN05_F32;
     }
   }
   if (g_mainloop == SAGE_MAINLOOP_DEFAULT) return tc_available() ? SAGE_MAINLOOP_TCGEN05 : SAGE_MAINLOOP_MMA_SYNC;
@@ -143,7 +144,11 @@ AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const i
 }
 
 int run_mainloop(const AttnParams& p, cudaStream_t s) {
-  return resolved_mainloop() == SAGE_MAINLOOP_TCGEN05 ? launch_attn_tc(p, s) : launch_attn_mma(p, s);
+  switch (resolved_mainloop()) {
+    case SAGE_MAINLOOP_TCGEN05: return launch_attn_tc(p, s);
+    case SAGE_MAINLOOP_TCGEN05_F32: return launch_attn_tc_f32(p, s);
+    default: return launch_attn_mma(p, s);
+  }
 }
 
 }  // namespace
@@ -282,7 +287,7 @@ const char* sage_strerror(int code) {
 }
 
 int sage_set_mainloop(int which) {
-  if (which < SAGE_MAINLOOP_DEFAULT || which > SAGE_MAINLOOP_MMA_SYNC) return SAGE_ERR_UNSUPPORTED;
+  if (which < SAGE_MAINLOOP_DEFAULT || which > SAGE_MAINLOOP_TCGEN05_F32) return SAGE_ERR_UNSUPPORTED;
   g_mainloop = which;
   g_mainloop_env_read = true;
   return SAGE_OK;
@@ -312,7 +317,7 @@ int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int 
   if ((rc = clear_status(workspace, s))) return rc;
   AttnParams p = make_params(d, q_i8, nullptr, k_i8, nullptr, nullptr, nullptr, nullptr, 0, 0, 0,
                              0.0f, workspace);
-  return resolved_mainloop() == SAGE_MAINLOOP_TCGEN05
+  return resolved_mainloop() != SAGE_MAINLOOP_MMA_SYNC  // both tcgen05 variants share the QK
              ? launch_debug_qk_tc(p, b, h, q_tile, k_tile, s_out, s)
              : launch_debug_qk_mma(p, b, h, q_tile, k_tile, s_out, s);
 }

@@ -110,6 +110,7 @@ int launch_attn_mma(const AttnParams& p, cudaStream_t s);
 int launch_debug_qk_mma(const AttnParams& p, int b, int h, int q_tile, int k_tile, int32_t* s_out,
                         cudaStream_t s);
 int launch_attn_tc(const AttnParams& p, cudaStream_t s);
+int launch_attn_tc_f32(const AttnParams& p, cudaStream_t s);
 int launch_debug_qk_tc(const AttnParams& p, int b, int h, int q_tile, int k_tile, int32_t* s_out,
                        cudaStream_t s);
 bool tc_available();

@@ -86,11 +86,22 @@ enum sage_op {
   SAGE_OP_DEBUG_QK = 4
 };
 
-/* Mainloop implementations (same numerics, chosen by measurement). */
+/* Mainloop implementations.  DEFAULT, TCGEN05 and MMA_SYNC compute the
+ * exact contract (same numerics, chosen by measurement).  TCGEN05_F32 is the
+ * fast variant the pages leave to a future backend with its own contract
+ * ("Vortex Exact", section "Scope"): same quantised inputs, INT8 QK^T and
+ * E4M3 probabilities, but the PV products accumulate in FP32 in TMEM across
+ * all tiles (no FP16 buffer per K32 slice) and the running maximum used for
+ * the probabilities is raised only when a tile's maximum exceeds it by more
+ * than 8 (log2 units), with the accumulator rescaled only then.  Its output
+ * is held to a quality gate (cosine similarity to FP64 attention, distance
+ * to the exact path), not to the oracle bit for bit.  It is never chosen by
+ * DEFAULT. */
 enum sage_mainloop {
-  SAGE_MAINLOOP_DEFAULT = 0, /* the fastest validated variant */
-  SAGE_MAINLOOP_TCGEN05 = 1, /* tcgen05 MMAs with TMEM accumulators, TMA */
-  SAGE_MAINLOOP_MMA_SYNC = 2 /* warp-level mma.sync */
+  SAGE_MAINLOOP_DEFAULT = 0,     /* the fastest validated exact variant */
+  SAGE_MAINLOOP_TCGEN05 = 1,     /* tcgen05 MMAs with TMEM accumulators, TMA */
+  SAGE_MAINLOOP_MMA_SYNC = 2,    /* warp-level mma.sync */
+  SAGE_MAINLOOP_TCGEN05_F32 = 3  /* quality-gated fast variant (see above) */
 };
 
 /* Bytes at the start of every workspace that hold the device status word. */

@@ -78,6 +78,12 @@ def test_argument_errors_need_no_device(lib):
     assert fq(None, 4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
     assert fq(4096, 4096, 4096 + 8, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_set_mainloop(7) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_set_mainloop(-1) == sage.SAGE_ERR_UNSUPPORTED
+    # every declared mainloop value is accepted; the explicit ones read back as set
+    for which in (sage.SAGE_MAINLOOP_TCGEN05, sage.SAGE_MAINLOOP_MMA_SYNC, sage.SAGE_MAINLOOP_TCGEN05_F32):
+        assert lib.sage_set_mainloop(which) == sage.SAGE_OK
+        assert lib.sage_get_mainloop() == which
+    assert lib.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT) == sage.SAGE_OK
     assert lib.sage_debug_qk_s32(4096, 4096, 1, 100, 2, 64, 0, 2, 0, 0, 4096, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
 
 

@@ -394,7 +394,7 @@ def main():
                          "traffic": recorded_traffic(cfg.name, ml_name)},
             "e2e": {"value": whole_job_tops(cfg.ops, world, e2e_ms), "unit": UNIT,
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * 8,
+            "gpu_launches": args.steps * 8,  # seven prepass kernels and the mainloop
             "clocks": clk.summary(),
         }
         if not args.no_cpu_baseline:

@@ -61,7 +61,7 @@ int check_out(const void* out, int64_t sb, int64_t sn, int64_t sh) {
 struct Layout {
   size_t status = 0;
   size_t q8 = 0, q_scale = 0, k8 = 0, k_scale = 0, k_mean = 0, v8 = 0, v_scale = 0;
-  size_t k_part = 0, v_part = 0, v_amax = 0;
+  size_t k_part = 0, v_part = 0, v_amax = 0, counters = 0;
   size_t total = 0;
 };
 
@@ -83,11 +83,13 @@ Layout plan(int op, const Dims& d) {
     L.v8 = take(bh * d.D * d.Nk);
     L.v_scale = take(bh * d.D * sizeof(float));
   }
-  if (op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
-  if (op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_V) {
+  const bool all3 = op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QKV;
+  if (all3 || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
+  if (all3 || op == SAGE_OP_QUANT_V) {
     L.v_part = take(bh * d.T64 * d.D * sizeof(float));
     L.v_amax = take(bh * d.D * sizeof(float));
   }
+  if (op == SAGE_OP_QUANT_QKV) L.counters = take((1 + 2 * bh) * sizeof(int));
   L.total = off;
   return L;
 }
@@ -102,6 +104,19 @@ int check_ws(void* ws, size_t bytes, size_t need) {
 template <class T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+FusedOut fused_out(void* ws, const Layout& L, int8_t* q8, float* qs, int8_t* k8, float* ks, float* km,
+                   uint8_t* v8, float* vs) {
+  FusedOut o;
+  o.q8 = q8; o.q_scale = qs; o.k8 = k8; o.k_scale = ks; o.k_mean = km; o.v8 = v8; o.v_scale = vs;
+  o.v_amax = at<float>(ws, L.v_amax);
+  o.k_part = at<double>(ws, L.k_part);
+  o.v_part = at<float>(ws, L.v_part);
+  o.counters = at<int>(ws, L.counters);
+  o.status = static_cast<DeviceStatus*>(ws);
+  o.wait_limit = g_wait_limit;
+  return o;
 }
 
 int clear_status(void* ws, cudaStream_t s) {
@@ -156,7 +171,7 @@ int run_mainloop(const AttnParams& p, cudaStream_t s) {
 extern "C" {
 
 int sage_workspace_bytes(int op, int B, int N, int H, int D, size_t* bytes) {
-  if (!bytes || op < SAGE_OP_QUANT_QK || op > SAGE_OP_DEBUG_QK) return SAGE_ERR_INVALID_ARG;
+  if (!bytes || op < SAGE_OP_QUANT_QK || op > SAGE_OP_QUANT_QKV) return SAGE_ERR_INVALID_ARG;
   int rc = check_dims(B, N, H, D);
   if (rc) return rc;
   *bytes = plan(op, make_dims(B, N, H, D)).total;
@@ -210,6 +225,26 @@ int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, f
                           at<float>(workspace, L.v_amax), s);
 }
 
+int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, int N, int H, int D,
+                   int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                   uint8_t* v_fp8, float* v_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(q)) || (rc = check_view(k)) || (rc = check_view(v))) return rc;
+  if (!q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean || !v_fp8 || !v_scale) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(q_scale) || !aligned16(k_scale) ||
+      !aligned16(k_mean) || !aligned16(v_fp8) || !aligned16(v_scale))
+    return SAGE_ERR_UNSUPPORTED;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_QUANT_QKV, d);
+  if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  return launch_prepass_fused(q, k, v, B, N, H, D,
+                              fused_out(workspace, L, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale), s);
+}
+
 int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
                          const float* k_scale, const uint8_t* v_fp8, const float* v_scale,
                          void* out, int64_t out_stride_b, int64_t out_stride_n,
@@ -253,6 +288,7 @@ int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* ou
   float* km = at<float>(workspace, L.k_mean);
   uint8_t* v8 = at<uint8_t>(workspace, L.v8);
   float* vs = at<float>(workspace, L.v_scale);
+  // the separate prepass kernels: faster than the single-launch one (measured)
   if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
     return rc;
   if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_part),

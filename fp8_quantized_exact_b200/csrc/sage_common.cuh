@@ -101,6 +101,24 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_
 
 // Host-side launchers (defined in the .cu files).
 namespace sage {
+// Outputs and scratch of the single-launch prepass (device pointers).
+struct FusedOut {
+  int8_t* q8;
+  float* q_scale;
+  int8_t* k8;
+  float* k_scale;
+  float* k_mean;
+  uint8_t* v8;
+  float* v_scale;
+  float* v_amax;       // [B][H][D]
+  double* k_part;      // [B][H][T64][D]
+  float* v_part;       // [B][H][T64][D]
+  int* counters;       // 1 + 2*B*H ints, zeroed by the launcher
+  DeviceStatus* status;
+  long long wait_limit;
+};
+int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
+                         int H, int D, const FusedOut& o, cudaStream_t s);
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
                       double* k_part, cudaStream_t s);

@@ -83,7 +83,8 @@ enum sage_op {
   SAGE_OP_QUANT_V = 1,
   SAGE_OP_ATTN_FWD = 2,
   SAGE_OP_ATTN_FROM_QUANT = 3,
-  SAGE_OP_DEBUG_QK = 4
+  SAGE_OP_DEBUG_QK = 4,
+  SAGE_OP_QUANT_QKV = 5
 };
 
 /* Mainloop implementations.  DEFAULT, TCGEN05 and MMA_SYNC compute the
@@ -135,6 +136,22 @@ SAGE_API int sage_quant_qk(sage_view_bf16 q, sage_view_bf16 k, int B, int N, int
 SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, float* v_scale,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* All three prepasses in one launch: the outputs of sage_quant_qk and
+ * sage_quant_v, bit for bit (same K sum order, same rounding).  Each head's
+ * K and V are read from HBM once; the quantisation re-reads them from L2
+ * (the pages' producer fusions, "Sage2 Blackwell Mainloop", section
+ * "Completed P1 And P2").  A persistent kernel takes work in head-major
+ * order; the K/V quantisation of a head waits, bounded, for the head's
+ * statistics (a wait that runs out leaves SAGE_ERR_TIMEOUT in the status
+ * word).  On one B200 it is slower than the two separate calls (1.75 ms
+ * against 1.21 ms at B1 N37810 H56 D128), which keep more memory streams in
+ * flight; sage_attn_fwd uses the separate kernels.
+ * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QKV, ...), 256-byte
+ * aligned; concurrent calls need separate workspaces. */
+SAGE_API int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, int N, int H, int D,
+                   int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                   uint8_t* v_fp8, float* v_scale, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Fused mainloop on quantised inputs: every 64-key tile in increasing order,
  * INT8 QK^T, score scaling, online softmax, E4M3 P, two K32 FP16 PV buffers
  * added into FP32, then 1/d, V scale and the BF16 store to `out`
@@ -149,8 +166,9 @@ SAGE_API int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, cons
                          int64_t out_stride_h, int B, int N, int H, int D, float sm_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
-/* The whole path: both prepasses (quantised tensors kept in the workspace)
- * then the fused mainloop.  Workspace: sage_workspace_bytes(
+/* The whole path: both prepasses (the separate kernels of sage_quant_qk and
+ * sage_quant_v; quantised tensors kept in the workspace) then the fused
+ * mainloop.  Workspace: sage_workspace_bytes(
  * SAGE_OP_ATTN_FWD, ...) bytes, 256-byte aligned. */
 SAGE_API int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* out,
                   int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N,

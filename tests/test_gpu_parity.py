@@ -153,6 +153,48 @@ def test_explicit_prepass_and_from_quant(sage, dev):
         assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
+def _quant_buffers(sage, B, N, H, D, dev, fill):
+    shp = sage.quant_shapes(B, N, H, D)
+    return {n: torch.full(s, fill, dtype=dt, device=dev) for (n, s), dt in zip(
+        shp.items(), (torch.int8, torch.float32, torch.int8, torch.float32, torch.float32,
+                      torch.uint8, torch.float32))}
+
+
+@pytest.mark.parametrize("shape,cfg", [((1, 1000, 3, 128), None), ((2, 333, 3, 64), None),
+                                       ((1, 65, 2, 128), None), ((1, 1, 1, 64), None),
+                                       (None, "ragged"), (None, "fused_small")])
+def test_single_launch_prepass_matches_separate(sage, dev, shape, cfg):
+    """sage_quant_qkv (one persistent launch) writes the same bytes, scales
+    and K mean as sage_quant_qk + sage_quant_v, padding included, and the
+    oracle's (bit-exact), on contiguous and fused-projection strides."""
+    if cfg == "fused_small":
+        inp = synth.make_inputs(synth.Config("fused_small", 1, 777, 4, 128, layout="fused_qkv"), seed=4)
+    elif cfg is not None:
+        inp = synth.make_inputs(synth.CONFIGS[cfg], seed=4)
+    else:
+        inp = synth.custom(*shape, seed=sum(shape))
+    B, N, H, D = inp.q.shape
+    (q, k, v), _ = gu.to_device(inp, dev)
+    a = _quant_buffers(sage, B, N, H, D, dev, 7)
+    b = _quant_buffers(sage, B, N, H, D, dev, 9)
+    sage.sage_quant_qkv(q, k, v, a["q_i8"], a["q_scale"], a["k_i8"], a["k_scale"], a["k_mean"],
+                        a["v_fp8"], a["v_scale"], sage.workspace(sage.SAGE_OP_QUANT_QKV, B, N, H, D, dev))
+    sage.sage_quant_qk(q, k, b["q_i8"], b["q_scale"], b["k_i8"], b["k_scale"], b["k_mean"],
+                       sage.workspace(sage.SAGE_OP_QUANT_QK, B, N, H, D, dev))
+    sage.sage_quant_v(v, b["v_fp8"], b["v_scale"], sage.workspace(sage.SAGE_OP_QUANT_V, B, N, H, D, dev))
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    qz = oracle.quantize(inp.q, inp.k, inp.v)
+    got = {"q8": a["q_i8"].cpu().numpy()[:, :, :N], "k8": a["k_i8"].cpu().numpy()[:, :, :N],
+           "v8": a["v_fp8"].cpu().numpy()[:, :, :, :N].transpose(0, 1, 3, 2),
+           "q_scale": a["q_scale"].cpu().numpy(), "k_scale": a["k_scale"].cpu().numpy(),
+           "k_mean": a["k_mean"].cpu().numpy(), "v_scale": a["v_scale"].cpu().numpy(),
+           "q_pad": a["q_i8"].cpu().numpy()[:, :, N:], "k_pad": a["k_i8"].cpu().numpy()[:, :, N:],
+           "v_pad": a["v_fp8"].cpu().numpy()[:, :, :, N:]}
+    check_quant(got, qz, N)
+
+
 def test_custom_softmax_scale(sage, dev):
     inp = synth.custom(1, 200, 2, 128, seed=21)
     (q, k, v), _ = gu.to_device(inp, dev)

@@ -66,6 +66,7 @@ def _lib(plant: int = 0):
         lib.oracle_quant_q.argtypes = strided + [_P, _P]
         lib.oracle_quant_k.argtypes = strided + [_P, _P, _P]
         lib.oracle_quant_v.argtypes = strided + [_P, _P]
+        lib.oracle_norm_rope.argtypes = strided + [_P, _P, _P, ctypes.c_float, _P]
         lib.oracle_attn_rows.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, ctypes.c_float,
                                          _I, _I, _I, _I, _P, _P]
         lib.oracle_qk_s32.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P]
@@ -144,6 +145,25 @@ def quant_v(v: np.ndarray, plant: int = 0):
     vs = np.zeros((B, H, D), np.float32)
     _ok(_lib(plant).oracle_quant_v(*_strided(v), _ptr(v8), _ptr(vs)))
     return v8, vs
+
+
+def norm_rope(x: np.ndarray, w: np.ndarray, cos_t: np.ndarray, sin_t: np.ndarray, eps: float,
+              plant: int = 0) -> np.ndarray:
+    """RMSNorm over D then split-half RoPE (reading R11) of a strided BF16
+    [B, N, H, D] view; weights BF16 bits [D], tables FP32 [N, D/2].  Returns
+    contiguous BF16 bits [B, N, H, D]."""
+    B, N, H, D = x.shape
+    z = np.zeros((B, N, H, D), np.uint16)
+    _ok(_lib(plant).oracle_norm_rope(*_strided(x), _ptr(np.ascontiguousarray(w, np.uint16)),
+                                     _ptr(np.ascontiguousarray(cos_t, np.float32)),
+                                     _ptr(np.ascontiguousarray(sin_t, np.float32)), float(eps), _ptr(z)))
+    return z
+
+
+def quantize_normed(q, k, v, wq, wk, cos_t, sin_t, eps, plant: int = 0) -> "Quantized":
+    """The producer (R11) on Q and K, then the same prepasses as quantize()."""
+    return quantize(norm_rope(q, wq, cos_t, sin_t, eps, plant), norm_rope(k, wk, cos_t, sin_t, eps, plant),
+                    v, plant)
 
 
 @dataclass

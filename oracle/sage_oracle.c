@@ -54,6 +54,17 @@
  *     instantaneous buffer: tmp = fp16_rne(exact sum of p8*v8), then
  *     RO = fl32(RO + float(tmp)) per slice, in slice order.
  *  R8 Output: rcp = fl32(1/d); out = bf16_rne(fl32(fl32(RO*rcp)*v_scale[d])).
+ *  R11 Q/K producer (RMSNorm + split-half RoPE before the Q/K quantisation;
+ *     "Sage2 Blackwell Mainloop", section "Completed P1 And P2", names the
+ *     fused producer but gives no formula or rounding).  Per (b, n, h) row x
+ *     of D BF16 values, BF16 weight w[D], FP32 tables cos/sin[N][D/2]:
+ *       ss = FP32 sum of fl32(x_d*x_d) in channel order;
+ *       r  = fl32(1 / fl32(sqrt(fl32(fl32(ss/D) + eps))))   (correctly rounded);
+ *       y_d = bf16(fl32(bf16(fl32(x_d*r)) * w_d));
+ *       for j < D/2, a = y_j, b = y_{j+D/2}, c = cos[n][j], s = sin[n][j]:
+ *         z_j       = bf16(fl32(fl32(a*c) - fl32(b*s))),
+ *         z_{j+D/2} = bf16(fl32(fl32(b*c) + fl32(a*s))).
+ *     z then goes through R1/R2 exactly as the raw Q and K do.
  *
  * Build: gcc -O2 -ffp-contract=off (no -ffast-math).  Defining
  * ORACLE_PLANT=<n> builds a deliberately wrong variant, used only by the
@@ -278,6 +289,45 @@ int oracle_quant_k(const uint16_t* k, int64_t sb, int64_t sn, int64_t sh, int B,
                        k8 + (((int64_t)b * H + h) * N + r0) * D,
                        &k_scale[((int64_t)b * H + h) * nt + t]);
       }
+  return ORACLE_OK;
+}
+
+/* ----------------------------------------- producer: RMSNorm + RoPE (R11)
+ * z[b][n][h][d] BF16 bits, contiguous, from the strided view x. */
+int oracle_norm_rope(const uint16_t* x, int64_t sb, int64_t sn, int64_t sh, int B, int N, int H, int D,
+                     const uint16_t* w, const float* cos_t, const float* sin_t, float eps, uint16_t* z) {
+  if (check_dims(B, N, H, D) || (D & 1) || !w || !cos_t || !sin_t || !z) return ORACLE_EINVAL;
+  const int half = D / 2;
+  float* y = (float*)malloc(sizeof(float) * (size_t)D);
+  if (!y) return ORACLE_ENOMEM;
+  for (int b = 0; b < B; ++b)
+    for (int n = 0; n < N; ++n)
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* row = x + b * sb + n * sn + h * sh;
+        float ss = 0.0f;
+        for (int d = 0; d < D; ++d) {
+          const float v = bf16_to_f32(row[d]);
+          ss = ss + v * v;
+        }
+        const float mean = ss / (float)D;
+        const float r = 1.0f / sqrtf(mean + eps);
+        for (int d = 0; d < D; ++d) {
+          const float xn = bf16_to_f32(f32_to_bf16(bf16_to_f32(row[d]) * r));
+          y[d] = bf16_to_f32(f32_to_bf16(xn * bf16_to_f32(w[d])));
+        }
+        uint16_t* out = z + (((size_t)b * N + n) * H + h) * D;
+        for (int j = 0; j < half; ++j) {
+          const float a = y[j], bb = y[j + half];
+          const float c = cos_t[(size_t)n * half + j], s = sin_t[(size_t)n * half + j];
+#if ORACLE_PLANT == 9
+          out[j] = f32_to_bf16(a * c + bb * s);      /* planted: rotation sign */
+#else
+          out[j] = f32_to_bf16(a * c - bb * s);
+#endif
+          out[j + half] = f32_to_bf16(bb * c + a * s);
+        }
+      }
+  free(y);
   return ORACLE_OK;
 }
 

@@ -314,6 +314,53 @@ def pin_qk_s32(plant=0):
     assert np.array_equal(S, ref)
 
 
+# ------------------------------------------- producer: RMSNorm + RoPE (R11)
+def _rope_tables(N, half, seed):
+    rng = np.random.default_rng(seed)
+    ang = rng.uniform(-np.pi, np.pi, (N, half))
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def pin_norm_rope_fp64(plant=0):
+    """Against RMSNorm and split-half RoPE written in float64 from their
+    definitions: within the three BF16 roundings of the reading."""
+    rng = np.random.default_rng(5)
+    N, H, D = 6, 2, 16
+    x = bf16_bits_round(rng.standard_normal((1, N, H, D)) * 1.7)
+    w = bf16_bits_round(rng.uniform(0.5, 1.5, D))
+    c, s_ = _rope_tables(N, D // 2, 6)
+    eps = 1e-6
+    z = synth.bf16_to_float(oracle.norm_rope(x, w, c, s_, eps, plant)).astype(np.float64)
+    X = synth.bf16_to_float(x).astype(np.float64)
+    W = synth.bf16_to_float(w).astype(np.float64)
+    y = X / np.sqrt((X * X).mean(axis=-1, keepdims=True) + eps) * W
+    a, b = y[..., : D // 2], y[..., D // 2:]
+    C, S = c.astype(np.float64)[None, :, None, :], s_.astype(np.float64)[None, :, None, :]
+    ref = np.concatenate([a * C - b * S, b * C + a * S], axis=-1)
+    scale = np.concatenate([np.abs(a) + np.abs(b)] * 2, axis=-1)
+    assert np.all(np.abs(z - ref) <= 2.0 ** -6 * scale + 1e-6), np.abs(z - ref).max()
+
+
+def pin_norm_rope_exact(plant=0):
+    """Closed forms: a constant row normalises to exactly +-1; a quarter turn
+    (cos 0, sin 1) swaps the halves with a sign; a weight of 2 doubles z."""
+    N, H, D = 3, 1, 8
+    ones_w = bf16_bits(np.ones(D, np.float32))
+    ident_c, ident_s = np.ones((N, D // 2), np.float32), np.zeros((N, D // 2), np.float32)
+    const = np.stack([np.full((H, D), v, np.float32) for v in (2.0, -0.5, 3.0)])[None]
+    z = synth.bf16_to_float(oracle.norm_rope(bf16_bits(const), ones_w, ident_c, ident_s, 1e-6, plant))
+    assert np.array_equal(z, np.sign(const)), z
+    rng = np.random.default_rng(8)
+    x = bf16_bits_round(rng.standard_normal((1, N, H, D)))
+    y = synth.bf16_to_float(oracle.norm_rope(x, ones_w, ident_c, ident_s, 1e-6, plant))
+    qt = synth.bf16_to_float(oracle.norm_rope(x, ones_w, np.zeros_like(ident_c), np.ones_like(ident_s), 1e-6, plant))
+    assert np.array_equal(qt[..., : D // 2], -y[..., D // 2:]) and np.array_equal(qt[..., D // 2:], y[..., : D // 2])
+    two = bf16_bits(np.full(D, 2.0, np.float32))
+    z2 = synth.bf16_to_float(oracle.norm_rope(x, two, ident_c, ident_s, 1e-6, plant))
+    assert np.array_equal(z2, 2.0 * y)
+
+
 ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_f16_round, pin_bf16_round, pin_worked_example,
             pin_group_boundaries, pin_q_zero_mean, pin_fp64_bruteforce, pin_dominance,
-            pin_k_offset_invariance, pin_denominator, pin_qk_s32]
+            pin_k_offset_invariance, pin_denominator, pin_qk_s32, pin_norm_rope_fp64,
+            pin_norm_rope_exact]

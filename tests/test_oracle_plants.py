@@ -14,6 +14,7 @@ PLANTS = {
     6: "old-max rescale of RO and d skipped",
     7: "max not subtracted before exp2",
     8: "V scale not applied in the epilogue",
+    9: "RoPE rotation sign flipped in the first half",
 }
 
 

@@ -40,7 +40,8 @@ SAGE_MAINLOOP_TCGEN05_F32 = 3  # quality-gated fast variant, not the exact contr
 SAGE_STATUS_BYTES = 256
 
 # every symbol the header declares (the CPU test checks the exports)
-EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_attn_from_quant",
+EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_norm_rope_quant_qk",
+           "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
            "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
            "sage_attn_fwd_noalloc", "sage_debug_set_stall")
@@ -81,6 +82,7 @@ def lib():
             "sage_quant_qk": [V, V, I, I, I, I, P, P, P, P, P, P, SZ, P],
             "sage_quant_v": [V, I, I, I, I, P, P, P, SZ, P],
             "sage_quant_qkv": [V, V, V, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P],
+            "sage_norm_rope_quant_qk": [V, V, P, P, P, P, ctypes.c_float, I, I, I, I, P, P, P, P, P, P, SZ, P],
             "sage_attn_from_quant": [P, P, P, P, P, P, P, L64, L64, L64, I, I, I, I,
                                      ctypes.c_float, P, SZ, P],
             "sage_attn_fwd": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P, SZ, P],
@@ -161,6 +163,16 @@ def sage_quant_qkv(q, k, v, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)),
            "sage_quant_qkv")
+
+
+def sage_norm_rope_quant_qk(q, k, wq, wk, cos_t, sin_t, eps, q_i8, q_scale, k_i8, k_scale, k_mean, workspace,
+                            stream=None):
+    B, N, H, D = q.shape
+    _check(lib().sage_norm_rope_quant_qk(_view(q), _view(k), _ptr(wq), _ptr(wk), _ptr(cos_t), _ptr(sin_t),
+                                         float(eps), B, N, H, D, _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                                         _ptr(k_scale), _ptr(k_mean), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)),
+           "sage_norm_rope_quant_qk")
 
 
 def sage_quant_v(v, v_fp8, v_scale, workspace, stream=None):

@@ -283,6 +283,10 @@ int prepass_v(const sage_view_bf16& v, int B, int N, int H, uint8_t* v8, float* 
 
 }  // namespace
 
+void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s) {
+  reduce_stats_kernel<true, false><<<BH, D, 0, s>>>(N, D, T64, k_part, k_mean, nullptr, nullptr, nullptr);
+}
+
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
                       double* k_part, cudaStream_t s) {

@@ -208,6 +208,29 @@ int sage_quant_qk(sage_view_bf16 q, sage_view_bf16 k, int B, int N, int H, int D
                            at<double>(workspace, L.k_part), s);
 }
 
+int sage_norm_rope_quant_qk(sage_view_bf16 q, sage_view_bf16 k, const void* wq, const void* wk, const float* cos_t,
+                            const float* sin_t, float eps, int B, int N, int H, int D, int8_t* q_i8, float* q_scale,
+                            int8_t* k_i8, float* k_scale, float* k_mean, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(q)) || (rc = check_view(k))) return rc;
+  if (!wq || !wk || !cos_t || !sin_t || !q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
+  if (!(eps >= 0.0f)) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(wq) || !aligned16(wk) || !aligned16(cos_t) || !aligned16(sin_t) || !aligned16(q_i8) ||
+      !aligned16(k_i8) || !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(k_mean))
+    return SAGE_ERR_UNSUPPORTED;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_QUANT_QK, d);
+  if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((rc = clear_status(workspace, s))) return rc;
+  NormRopeIn in{static_cast<const uint16_t*>(wq), static_cast<const uint16_t*>(wk), cos_t, sin_t, eps};
+  return launch_norm_rope_qk(in, q, k, B, N, H, D, q_i8, q_scale, k_i8, k_scale, k_mean,
+                             at<double>(workspace, L.k_part), s);
+}
+
 int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, float* v_scale,
                  void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_dims(B, N, H, D);

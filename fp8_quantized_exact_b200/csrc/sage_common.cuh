@@ -117,6 +117,18 @@ struct FusedOut {
   DeviceStatus* status;
   long long wait_limit;
 };
+// Inputs of the RMSNorm + RoPE producer (device pointers).
+struct NormRopeIn {
+  const uint16_t* wq;   // BF16 [D]
+  const uint16_t* wk;   // BF16 [D]
+  const float* cos_t;   // FP32 [N][D/2]
+  const float* sin_t;   // FP32 [N][D/2]
+  float eps;
+};
+int launch_norm_rope_qk(const NormRopeIn& in, const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H,
+                        int D, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean, double* k_part,
+                        cudaStream_t s);
+void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s);
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s);
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,

@@ -128,6 +128,23 @@ SAGE_API int sage_quant_qk(sage_view_bf16 q, sage_view_bf16 k, int B, int N, int
                   int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Q/K producer with RMSNorm and split-half RoPE in front of the quantisation
+ * (the fused strided-NHD producer of "Sage2 Blackwell Mainloop", section
+ * "Completed P1 And P2"): per (b, n, h) row x of D values,
+ *   ss = FP32 sum of fl32(x_d*x_d) in channel order,
+ *   r  = fl32(1 / fl32(sqrt(fl32(fl32(ss/D) + eps)))),
+ *   y_d = bf16(fl32(bf16(fl32(x_d*r)) * w_d)),
+ *   z_j = bf16(fl32(fl32(y_j*c) - fl32(y_{j+D/2}*s))),
+ *   z_{j+D/2} = bf16(fl32(fl32(y_{j+D/2}*c) + fl32(y_j*s))),  c, s = cos/sin[n][j];
+ * then z goes through exactly the rules of sage_quant_qk (same outputs and
+ * layouts).  wq, wk: BF16 [D]; cos_t, sin_t: FP32 [N][D/2] row-major; all
+ * 16-byte aligned; eps >= 0.  The normalised rows are not stored.
+ * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QK, ...). */
+SAGE_API int sage_norm_rope_quant_qk(sage_view_bf16 q, sage_view_bf16 k, const void* wq, const void* wk,
+                            const float* cos_t, const float* sin_t, float eps, int B, int N, int H, int D,
+                            int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Prepass for V: per-channel amax over all tokens, scale, E4M3 bytes stored
  * transposed.  Defined by "Sage2 Blackwell Mainloop", section "Decision"
  * (V transpose/pad/permute, V scale/FP8 quantization) and section

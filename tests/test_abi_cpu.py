@@ -77,6 +77,22 @@ def test_argument_errors_need_no_device(lib):
     fq = lib.sage_attn_from_quant
     assert fq(None, 4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
     assert fq(4096, 4096, 4096 + 8, 4096, 4096, 4096, 4096, 0, 0, 0, 1, 10, 2, 64, 0.0, 4096, 4096, None) == sage.SAGE_ERR_UNSUPPORTED
+    nr = lib.sage_norm_rope_quant_qk
+    v4 = sage.sage_view_bf16(4096, 0, 128, 128)
+    # (q, k, wq, wk, cos, sin, eps, B, N, H, D, q8, qs, k8, ks, km, ws, ws_bytes, stream)
+    assert nr(v4, v4, None, 4096, 4096, 4096, 1e-6, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+              None) == sage.SAGE_ERR_INVALID_ARG
+    assert nr(v4, v4, 4096, 4096, 4096, 4096, -1.0, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+              None) == sage.SAGE_ERR_INVALID_ARG
+    assert nr(v4, v4, 4096 + 2, 4096, 4096, 4096, 1e-6, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+              None) == sage.SAGE_ERR_UNSUPPORTED
+    assert nr(v4, v4, 4096, 4096, 4096, 4096, 1e-6, 1, 10, 2, 96, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+              None) == sage.SAGE_ERR_UNSUPPORTED
+    qkv = lib.sage_quant_qkv
+    assert qkv(v4, v4, v4, 1, 10, 2, 64, None, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+               None) == sage.SAGE_ERR_INVALID_ARG
+    assert qkv(v4, v4, v4, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 100,
+               None) == sage.SAGE_ERR_WORKSPACE
     assert lib.sage_set_mainloop(7) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_set_mainloop(-1) == sage.SAGE_ERR_UNSUPPORTED
     # every declared mainloop value is accepted; the explicit ones read back as set

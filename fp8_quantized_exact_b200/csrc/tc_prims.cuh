@@ -29,13 +29,10 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait.  Returns false if the CTA is aborting or the wait ran out
-// (then the status word and the abort flag are set).  A phase that is
-// already complete costs one try_wait.
-__device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                             DeviceStatus* st, int where, long long limit,
-                                             bool honour_abort = true) {
-  if (mbar_try(b, parity)) return true;
+// The slow path of a bounded wait, kept out of line: inlined at every wait
+// it made the mainloops' hot code several times larger.
+static __device__ __noinline__ bool wait_slow(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                              DeviceStatus* st, int where, long long limit, bool honour_abort) {
   const long long t0 = clock64();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try(b, parity)) return true;
@@ -50,6 +47,15 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volat
     st->block = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
   }
   return false;
+}
+// Bounded wait.  Returns false if the CTA is aborting or the wait ran out
+// (then the status word and the abort flag are set).  A phase that is
+// already complete costs one try_wait.
+__device__ __forceinline__ bool wait_bounded(uint64_t* b, uint32_t parity, volatile int* abort_flag,
+                                             DeviceStatus* st, int where, long long limit,
+                                             bool honour_abort = true) {
+  if (mbar_try(b, parity)) return true;
+  return wait_slow(b, parity, abort_flag, st, where, limit, honour_abort);
 }
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,

@@ -47,6 +47,8 @@
 // at the end; the pages leave its summation order open.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "sage_common.cuh"
 #include "tc_prims.cuh"
 
@@ -149,12 +151,15 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     const int ntail = p.N - (T - 1) * kKTile;  // valid keys of the last tile
     float m_own = -INFINITY, d_own = 0.0f;     // this warp's latest running max and partial denominator
     float ks_next = par < T ? ksc[par] : 0.0f;  // K scale of this warp's next tile, loaded a tile ahead
-    for (int t = par; t < T; t += 2) {
+    // one 64-key tile t of this warp (TAIL: the ragged last tile, keys >= ntail
+    // masked); returns false if a wait gave up
+    auto tile_step = [&](auto tail_tag, int t) -> bool {
+      constexpr bool TAIL = decltype(tail_tag)::value;
       const int g = t >> 1, sb = g & 1;
       const uint32_t cols = kColS + 128 * sb + 64 * par;
       const float ks = ks_next;
       if (t + 2 < T) ks_next = ksc[t + 2];
-      if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) break;
+      if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) return false;
       tc_fence_after();
       uint32_t S[64];
       tmem_ld64(lane_addr + cols, S);
@@ -163,14 +168,13 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const bool m_ready = t == 0 || mbar_try(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1));
       const bool r_ready = mbar_try(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1));
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
-      const bool tail = t + 1 == T && ntail != kKTile;
-      const float tmax = tail ? tile_max<true>(S, cs, ntail) : tile_max<false>(S, cs, kKTile);
+      const float tmax = tile_max<TAIL>(S, cs, ntail);
       // running max: m(t) = max(m(t-1), tile max), m(t-1) from the partner warp
       float m_prev = -INFINITY;
       if (t > 0) {
         if (!m_ready && !wait_bounded(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1), abort_flag,
                                       p.status, 15, p.wait_limit))
-          break;
+          return false;
         m_prev = sm.m_x[par ^ 1][i];
       }
       const float m_new = fmaxf(m_prev, tmax);
@@ -178,8 +182,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_arrive(&sm.m_full[quad][par]);
       const float r = (m_new == m_prev) ? 1.0f : ex2(__fsub_rn(m_prev, m_new));
       uint32_t P[16];
-      const float rs = tail ? tile_exp<true>(lane_addr + cols, cs, m_new, ntail, P)
-                            : tile_exp<false>(lane_addr + cols, cs, m_new, kKTile, P);
+      const float rs = tile_exp<TAIL>(lane_addr + cols, cs, m_new, ntail, P);
       // this warp's partial denominator, carried from its previous tile's max
       d_own = (m_own == m_new) ? __fadd_rn(d_own, rs) : __fadd_rn(__fmul_rn(d_own, ex2(__fsub_rn(m_own, m_new))), rs);
       m_own = m_new;
@@ -187,11 +190,19 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       tmem_wait_st();
       if (!r_ready &&
           !wait_bounded(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 2, p.wait_limit))
-        break;
+        return false;
       sm.r_ring[par][i] = r;
       tc_fence_before();
       mbar_arrive(&sm.p_full[par]);
-    }
+      return true;
+    };
+    // the loop holds one copy of the tile code; a ragged last tile is peeled
+    // off after it, so the masked copy stays out of the hot loop
+    const int t_full = ntail == kKTile ? T : T - 1;  // tiles without masking
+    bool ok = true;
+    int t = par;
+    for (; ok && t < t_full; t += 2) ok = tile_step(std::false_type{}, t);
+    if (ok && t == T - 1 && t_full < T) tile_step(std::true_type{}, t);
     // merge the two partial denominators at the final running max
     sm.m_fin[par][i] = m_own;
     sm.d_fin[par][i] = d_own;

@@ -33,6 +33,8 @@
 // issues; every wait is bounded as in the exact mainloop.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "sage_common.cuh"
 #include "tc_prims.cuh"
 
@@ -140,12 +142,13 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     const int ntail = p.N - (T - 1) * kKTile;
     float m_own = -INFINITY, d_own = 0.0f;  // this warp's latest used max and partial denominator
     float ks_next = par < T ? ksc[par] : 0.0f;
-    for (int t = par; t < T; t += 2) {
+    auto tile_step = [&](auto tail_tag, int t) -> bool {
+      constexpr bool TAIL = decltype(tail_tag)::value;
       const int g = t >> 1, sb = g & 1;
       const uint32_t cols = kColSF + 128 * sb + 64 * par;
       const float ks = ks_next;
       if (t + 2 < T) ks_next = ksc[t + 2];
-      if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) break;
+      if (!wait_bounded(&sm.s_full[sb], (uint32_t)((g >> 1) & 1), abort_flag, p.status, 1, p.wait_limit)) return false;
       tc_fence_after();
       uint32_t S[64];
       tmem_ld64(lane_addr + cols, S);
@@ -153,15 +156,14 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const bool m_ready = t == 0 || __all_sync(0xffffffffu, mbar_try(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1)));
       const bool r_ready = __all_sync(0xffffffffu, mbar_try(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1)));
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
-      const bool tail = t + 1 == T && ntail != kKTile;
-      const float tmax = tail ? tile_max<true>(S, cs, ntail) : tile_max<false>(S, cs, kKTile);
+      const float tmax = tile_max<TAIL>(S, cs, ntail);
       // used max: raised to the tile max only when that exceeds it by more
       // than kRescaleLog2, so every p = 2^(s - m) stays <= 2^kRescaleLog2
       float m_prev = -INFINITY;
       if (t > 0) {
         if (!m_ready && !wait_bounded(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1), abort_flag,
                                       p.status, 15, p.wait_limit))
-          break;
+          return false;
         m_prev = sm.m_x[par ^ 1][i];
       }
       const float m_new = tmax > m_prev + kRescaleLog2 ? tmax : m_prev;
@@ -170,8 +172,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       // the accumulator is empty before tile 0, so nothing is rescaled there
       const float r = (t == 0 || m_new == m_prev) ? 1.0f : ex2(__fsub_rn(m_prev, m_new));
       uint32_t P[16];
-      const float rs = tail ? tile_exp<true>(lane_addr + cols, cs, m_new, ntail, P)
-                            : tile_exp<false>(lane_addr + cols, cs, m_new, kKTile, P);
+      const float rs = tile_exp<TAIL>(lane_addr + cols, cs, m_new, ntail, P);
       d_own = (m_own == m_new) ? __fadd_rn(d_own, rs) : __fadd_rn(__fmul_rn(d_own, ex2(__fsub_rn(m_own, m_new))), rs);
       m_own = m_new;
       tmem_st16(lane_addr + cols, P);
@@ -179,12 +180,19 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       const bool need = __any_sync(0xffffffffu, r != 1.0f);
       if (!r_ready &&
           !wait_bounded(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1), abort_flag, p.status, 2, p.wait_limit))
-        break;
+        return false;
       sm.r_ring[par][i] = r;
       if (lane == 0) sm.corr[par][quad] = need ? 1 : 0;
       tc_fence_before();
       mbar_arrive(&sm.p_full[par]);
-    }
+      return true;
+    };
+    // one copy of the tile code in the loop; a ragged last tile is peeled off
+    const int t_full = ntail == kKTile ? T : T - 1;
+    bool ok = true;
+    int t = par;
+    for (; ok && t < t_full; t += 2) ok = tile_step(std::false_type{}, t);
+    if (ok && t == T - 1 && t_full < T) tile_step(std::true_type{}, t);
     sm.m_fin[par][i] = m_own;
     sm.d_fin[par][i] = d_own;
     mbar_arrive(&sm.fin);

@@ -36,7 +36,13 @@ METRIC = ("sage_attn_fwd effective TOPS (4*B*H*N^2*D / step time) at N=37810, H=
 UNIT = "TOPS"
 NOMINAL_I8_OVER_BF16 = 2.0        # dense INT8/FP8 : BF16 tensor peak (4.5 : 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0     # used only when MEASURED_PEAKS.json is absent
-MAINLOOP_SOURCES = ["attn_tc.cu", "attn_mma.cu", "attn_tc_f32.cu", "tc_prims.cuh", "sage_common.cuh"]
+# the sources each mainloop kernel is compiled from (a recorded traffic figure
+# is valid only for the kernel source it was taken on)
+MAINLOOP_SOURCES = {
+    "tcgen05": ["attn_tc.cu", "tc_prims.cuh", "sage_common.cuh"],
+    "tcgen05_f32": ["attn_tc_f32.cu", "tc_prims.cuh", "sage_common.cuh"],
+    "mma_sync": ["attn_mma.cu", "sage_common.cuh"],
+}
 
 
 def parse():
@@ -62,9 +68,9 @@ def peaks():
     return FALLBACK_BF16_TFLOPS, 1400.0, 6650.0, "fallback"
 
 
-def kernel_hash():
+def kernel_hash(mainloop: str):
     h = hashlib.sha256()
-    for fn in MAINLOOP_SOURCES:
+    for fn in MAINLOOP_SOURCES[mainloop]:
         p = os.path.join(ROOT, "fp8_quantized_exact_b200", "csrc", fn)
         if os.path.exists(p):
             h.update(open(p, "rb").read())
@@ -80,7 +86,7 @@ def recorded_traffic(workload: str, mainloop: str):
     try:
         rec = json.load(open(path))
         e = rec.get(workload, {}).get(mainloop)
-        if e and e.get("kernel_hash") == kernel_hash():
+        if e and e.get("kernel_hash") == kernel_hash(mainloop):
             return e.get("dram_bytes_per_launch")
     except Exception:
         return None
@@ -336,6 +342,10 @@ def main():
         t1.record(stream)
         torch.cuda.synchronize()
         barrier()
+    for w in (ws_qk, ws_v, ws_m):
+        st = sage.sage_read_device_status(w)
+        if st != sage.SAGE_OK:
+            raise RuntimeError(f"device status after the timed steps: {sage.sage_strerror(st)}")
     total_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     ml_ms = [a.elapsed_time(b) for _, a, b in evs]
     step_ms = [s0.elapsed_time(b) for s0, _, b in evs]

@@ -69,7 +69,7 @@ struct F32Smem {
   uint64_t kv_full[kStagesF], kv_empty[kStagesF];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_acc;          // completes once per tile when that tile's PV MMAs are done
+  uint64_t o_acc[4];       // o_acc[t & 3] completes when the PV MMAs of tile t are done
   uint64_t c_done;         // completes once per rescaled tile when the accumulator is scaled
   uint64_t m_full[4][2];
   uint64_t fin, done;
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       mbar_init(&sm.r_free[i], kQTile + 1);  // correction owners and the PV issuer
       for (int q = 0; q < 4; ++q) mbar_init(&sm.m_full[q][i], 32);
     }
-    mbar_init(&sm.o_acc, 1);
+    for (int j = 0; j < 4; ++j) mbar_init(&sm.o_acc[j], 1);
     mbar_init(&sm.c_done, kQTile);
     mbar_init(&sm.fin, 2 * kQTile);
     mbar_init(&sm.done, kQTile);
@@ -214,16 +214,23 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
-      // follow the accumulator phase by phase: PV(t - 1) has completed, so the
-      // accumulator holds tiles 0 .. t-1 (and the parity below is unambiguous)
-      if (t > 0 && !wait_bounded(&sm.o_acc, (uint32_t)((t - 1) & 1), abort_flag, p.status, 20, p.wait_limit)) break;
+      // PV(t - 1) has completed, so the accumulator holds tiles 0 .. t-1.  The
+      // parity is unambiguous: this warp saw tile t - 5 complete on the same
+      // barrier, and the next MMAs that complete it, PV(t + 3), need the
+      // probabilities of tile t + 3, which wait for this warp's r_free
+      // arrival for tile t + 1.
+      if (t > 0 && !wait_bounded(&sm.o_acc[(t - 1) & 3], (uint32_t)(((t - 1) >> 2) & 1), abort_flag, p.status, 20,
+                                 p.wait_limit))
+        break;
       if (!wait_bounded(&sm.p_full[bi], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 3, p.wait_limit)) break;
+      // r and the flags are read before the arrival: after it the softmax
+      // owners of tile t + 2 may overwrite them
       const float r = sm.r_ring[bi][i];
       const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&sm.corr[bi][0]);
       mbar_arrive(&sm.r_free[bi]);
       if (flags == 0) continue;
       // every quadrant takes part, so c_done completes once per rescaled tile
-      if (sm.corr[bi][quad]) {
+      if ((flags >> (8 * quad)) & 0xFFu) {
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 64) {
@@ -240,7 +247,8 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       mbar_arrive(&sm.c_done);
     }
     // epilogue: the last PV MMAs have completed and 1/d is known
-    if (ok && T > 0 && wait_bounded(&sm.o_acc, (uint32_t)((T - 1) & 1), abort_flag, p.status, 21, p.wait_limit) &&
+    if (ok && T > 0 &&
+        wait_bounded(&sm.o_acc[(T - 1) & 3], (uint32_t)(((T - 1) >> 2) & 1), abort_flag, p.status, 21, p.wait_limit) &&
         wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) && !*abort_flag) {
       tc_fence_after();
       const int row = qt * kQTile + i;
@@ -334,8 +342,9 @@ __global__ void __launch_bounds__(kThreadsF, 1)
                  wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStagesF) & 1), abort_flag, p.status, 18, p.wait_limit));
       __syncwarp();
       if (!ok) break;
-      // a rescaled tile waits until the correction owners have scaled the accumulator
-      const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&sm.corr[half][0]);
+      // a rescaled tile waits until the correction owners have scaled the
+      // accumulator; lane 0's reading of the flags decides for the warp
+      const uint32_t flags = __shfl_sync(0xffffffffu, *reinterpret_cast<volatile uint32_t*>(&sm.corr[half][0]), 0);
       if (flags != 0) {
         ok = wait_bounded(&sm.c_done, (uint32_t)(ncorr & 1), abort_flag, p.status, 19, p.wait_limit);
         __syncwarp();
@@ -350,7 +359,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
         for (int sl = 0; sl < 2; ++sl)
           mma_f8_ts(tmem + kColOF, tmem + kColSF + 128 * sb + 64 * half + 8 * sl, vdesc + 2 * sl, ipv,
                     (t > 0 || sl > 0) ? 1u : 0u);
-        tc_commit(&sm.o_acc);
+        tc_commit(&sm.o_acc[t & 3]);
         if (half == 1 || t + 1 == T) {
           tc_commit(&sm.s_free[sb]);
           tc_commit(&sm.kv_empty[st]);

@@ -151,36 +151,38 @@ __global__ void __launch_bounds__(128) quant_q_kernel(const uint16_t* __restrict
   }
 }
 
-// K: one 128-thread block per 64-row block; x' = fl32(x - k_mean[d]).
+// K: one 128-thread block per 64-row block; x' = fl32(x - k_mean[d]).  The
+// raw BF16 chunks stay in registers between the amax pass and the code pass
+// (x' is recomputed, the same single rounding), which keeps the block small
+// enough for many blocks per SM.
 template <int D>
-__global__ void __launch_bounds__(128) quant_k_kernel(const uint16_t* __restrict__ k, int64_t sb,
-                                                      int64_t sn, int64_t sh, int N, int H, int Nk,
-                                                      int T64, const float* __restrict__ k_mean,
-                                                      int8_t* __restrict__ k8,
-                                                      float* __restrict__ k_scale) {
+__global__ void __launch_bounds__(128, 8) quant_k_kernel(const uint16_t* __restrict__ k, int64_t sb,
+                                                         int64_t sn, int64_t sh, int N, int H, int Nk,
+                                                         int T64, const float* __restrict__ k_mean,
+                                                         int8_t* __restrict__ k8,
+                                                         float* __restrict__ k_scale) {
   constexpr int SEG = D / 8;
   constexpr int PER = kKTile * SEG / 128;
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int col = (threadIdx.x % SEG) * 8;
+  uint4 xr[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int row = t * kKTile + (threadIdx.x + 128 * i) / SEG;
+    xr[i] = row < N ? ldg16(k + b * sb + (int64_t)row * sn + h * sh + col) : make_uint4(0, 0, 0, 0);
+  }
   float km[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) km[j] = k_mean[(size_t)(b * H + h) * D + col + j];
-  float xs[PER][8];
+  for (int j = 0; j < 8; ++j) km[j] = __ldg(k_mean + (size_t)(b * H + h) * D + col + j);
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int row = t * kKTile + (threadIdx.x + 128 * i) / SEG;
     if (row < N) {
       float f[8];
-      unpack_bf16x8(ldg16(k + b * sb + (int64_t)row * sn + h * sh + col), f);
+      unpack_bf16x8(xr[i], f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        xs[i][j] = __fsub_rn(f[j], km[j]);
-        amax = fmaxf(amax, fabsf(xs[i][j]));
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) xs[i][j] = 0.0f;
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fsub_rn(f[j], km[j])));
     }
   }
   __shared__ float red[4];
@@ -194,53 +196,82 @@ __global__ void __launch_bounds__(128) quant_k_kernel(const uint16_t* __restrict
   int8_t* dst = k8 + ((size_t)(b * H + h) * Nk + (size_t)t * kKTile) * D;
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
-    const int row = (threadIdx.x + 128 * i) / SEG;
-    uint2 o;
-    o.x = i8_code(xs[i][0], inv) | i8_code(xs[i][1], inv) << 8 | i8_code(xs[i][2], inv) << 16 |
-          i8_code(xs[i][3], inv) << 24;
-    o.y = i8_code(xs[i][4], inv) | i8_code(xs[i][5], inv) << 8 | i8_code(xs[i][6], inv) << 16 |
-          i8_code(xs[i][7], inv) << 24;
-    *reinterpret_cast<uint2*>(dst + (size_t)row * D + col) = o;
+    const int r = (threadIdx.x + 128 * i) / SEG;
+    uint2 o = make_uint2(0u, 0u);  // pad rows get zero codes
+    if (t * kKTile + r < N) {
+      float f[8];
+      unpack_bf16x8(xr[i], f);
+      float x[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) x[j] = __fsub_rn(f[j], km[j]);
+      o.x = i8_code(x[0], inv) | i8_code(x[1], inv) << 8 | i8_code(x[2], inv) << 16 | i8_code(x[3], inv) << 24;
+      o.y = i8_code(x[4], inv) | i8_code(x[5], inv) << 8 | i8_code(x[6], inv) << 16 | i8_code(x[7], inv) << 24;
+    }
+    *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
   }
 }
 
-// V: one thread per pair of channels of one 64-token chunk; the E4M3 bytes
-// are transposed in registers (token t of channel d goes to byte t of the
-// channel's 64-byte row) and stored as four 16-byte vectors per channel.
+// V: one 256-thread block per 128 tokens of one head.  The BF16 rows are
+// staged in shared memory with 16-byte loads; the 16-byte chunk index of a
+// row is XORed with bits 4-5 of its token, so that the column reads below
+// (four 16-token runs x eight channels per warp) fall in distinct banks.
+// Each thread then converts 16 consecutive tokens of one channel to E4M3
+// (two tokens per conversion, the earlier token in the low byte, so token t
+// is byte t of the channel's row) and writes them as one 16-byte vector; a
+// warp writes eight channels x 64 contiguous bytes.
+constexpr int kVTokens = 2 * kKTile;  // tokens per quant_v block
+
 template <int D>
-__global__ void __launch_bounds__(D / 2) quant_v_kernel(const uint16_t* __restrict__ v, int64_t sb,
-                                                        int64_t sn, int64_t sh, int N, int H,
-                                                        int Nk, const float* __restrict__ v_amax,
-                                                        uint8_t* __restrict__ v8) {
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int d0 = threadIdx.x * 2;
-  const float a0 = v_amax[(size_t)(b * H + h) * D + d0];
-  const float a1 = v_amax[(size_t)(b * H + h) * D + d0 + 1];
-  const float inv0 = a0 > 0.0f ? __fdiv_rn(448.0f, a0) : 0.0f;
-  const float inv1 = a1 > 0.0f ? __fdiv_rn(448.0f, a1) : 0.0f;
-  uint32_t w0[16], w1[16];  // 64 bytes per channel
+__global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ v, int64_t sb,
+                                                      int64_t sn, int64_t sh, int N, int H, int Nk,
+                                                      const float* __restrict__ v_amax,
+                                                      uint8_t* __restrict__ v8) {
+  constexpr int SEG = D / 8;                   // 16-byte chunks per token row
+  constexpr int LOADS = kVTokens * SEG / 256;  // chunks staged per thread
+  constexpr int RUNS = D * (kVTokens / 16) / 256;  // 16-token runs converted per thread
+  __shared__ __align__(16) uint4 tile[kVTokens * SEG];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int n0 = blockIdx.x * kVTokens;
+  const uint16_t* vp = v + b * sb + h * sh;
+  uint4 x[LOADS];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) { w0[i] = 0u; w1[i] = 0u; }
-  const uint16_t* vp = v + b * sb + h * sh + d0;
-#pragma unroll
-  for (int t = 0; t < kKTile; ++t) {
-    const int n = c * kKTile + t;
-    if (n < N) {
-      const uint32_t pair = __ldg(reinterpret_cast<const uint32_t*>(vp + (int64_t)n * sn));
-      const float x0 = __uint_as_float(pair << 16), x1 = __uint_as_float(pair & 0xFFFF0000u);
-      const uint16_t e = e4m3x2(__fmul_rn(x0, inv0), __fmul_rn(x1, inv1));
-      const uint32_t b0 = a0 > 0.0f ? (e & 0xFFu) : 0u;
-      const uint32_t b1 = a1 > 0.0f ? (e >> 8) : 0u;
-      w0[t >> 2] |= b0 << (8 * (t & 3));
-      w1[t >> 2] |= b1 << (8 * (t & 3));
-    }
+  for (int i = 0; i < LOADS; ++i) {
+    const int idx = threadIdx.x + 256 * i;
+    const int r = idx / SEG, k = idx % SEG;
+    x[i] = n0 + r < N ? ldg16(vp + (int64_t)(n0 + r) * sn + k * 8) : make_uint4(0, 0, 0, 0);
   }
-  uint8_t* r0 = v8 + ((size_t)(b * H + h) * D + d0) * Nk + (size_t)c * kKTile;
-  uint8_t* r1 = r0 + Nk;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    reinterpret_cast<uint4*>(r0)[i] = make_uint4(w0[4 * i], w0[4 * i + 1], w0[4 * i + 2], w0[4 * i + 3]);
-    reinterpret_cast<uint4*>(r1)[i] = make_uint4(w1[4 * i], w1[4 * i + 1], w1[4 * i + 2], w1[4 * i + 3]);
+  for (int i = 0; i < LOADS; ++i) {
+    const int idx = threadIdx.x + 256 * i;
+    const int r = idx / SEG, k = idx % SEG;
+    tile[r * SEG + (k ^ ((r >> 4) & 3))] = x[i];
+  }
+  __syncthreads();
+  const uint16_t* ts = reinterpret_cast<const uint16_t*>(tile);
+  const float* am = v_amax + (size_t)(b * H + h) * D;
+#pragma unroll
+  for (int i = 0; i < RUNS; ++i) {
+    const int idx = threadIdx.x + 256 * i;
+    const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
+    const int cb = rest % SEG, half = rest / SEG;
+    const int t0 = half * kKTile + 16 * q;  // first token of the run; (t >> 4) & 3 == q
+    if (n0 + half * kKTile >= Nk) continue;  // past the padded length
+    const int ch = cb * 8 + cl;
+    const float a = am[ch];
+    const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+    const uint16_t* col = ts + (cb ^ q) * 8 + cl;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int t = t0 + 4 * j;
+      const uint32_t lo = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[t * D]), inv),
+                                 __fmul_rn(bf16_bits_to_f32(col[(t + 1) * D]), inv));
+      const uint32_t hi = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[(t + 2) * D]), inv),
+                                 __fmul_rn(bf16_bits_to_f32(col[(t + 3) * D]), inv));
+      w[j] = a > 0.0f ? (lo | (hi << 16)) : 0u;
+    }
+    uint8_t* dst = v8 + ((size_t)(b * H + h) * D + ch) * Nk + n0 + t0;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -276,8 +307,8 @@ int prepass_v(const sage_view_bf16& v, int B, int N, int H, uint8_t* v8, float* 
       nullptr, 0, 0, 0, vp, v.stride_b, v.stride_n, v.stride_h, N, H, T64, nullptr, v_part);
   reduce_stats_kernel<false, true><<<B * H, D, 0, s>>>(N, D, T64, nullptr, nullptr, v_part, v_scale,
                                                        v_amax);
-  quant_v_kernel<D><<<dim3(T64, H, B), D / 2, 0, s>>>(vp, v.stride_b, v.stride_n, v.stride_h, N, H,
-                                                      Nk, v_amax, v8);
+  quant_v_kernel<D><<<dim3(ceil_div(Nk, kVTokens), H, B), 256, 0, s>>>(vp, v.stride_b, v.stride_n,
+                                                                       v.stride_h, N, H, Nk, v_amax, v8);
   return check_launch();
 }
 

@@ -151,3 +151,22 @@ def test_fast_repeat_is_deterministic(sage, dev):
     b, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05_F32)
     sage.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_fast_repeat_with_rescales_status_and_bits(sage, dev):
+    # hundreds of CTAs, each rescaling its accumulator on several tiles (the
+    # key scale doubles three times along the sequence), launched repeatedly:
+    # every launch must end with a clean status (no bounded wait ran out) and
+    # give the same bits
+    inp = synth.custom(1, 4096, 8, 128, seed=21, k_offset=0.0)
+    for start in (1024, 2048, 3072):
+        _scale_keys(inp, start, 2.0)
+    (q, k, v), _ = gu.to_device(inp, dev)
+    ref = None
+    for _ in range(8):
+        out, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05_F32)
+        if ref is None:
+            ref = out.clone()
+        else:
+            assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    sage.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT)

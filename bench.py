@@ -36,6 +36,7 @@ METRIC = ("sage_attn_fwd effective TOPS (4*B*H*N^2*D / step time) at N=37810, H=
 UNIT = "TOPS"
 NOMINAL_I8_OVER_BF16 = 2.0        # dense INT8/FP8 : BF16 tensor peak (4.5 : 2.25 PFLOP/s)
 FALLBACK_BF16_TFLOPS = 1590.0     # used only when MEASURED_PEAKS.json is absent
+REF_BUDGET_S = 120.0  # timed oracle seconds the reference arm aims for, all steps together
 # the sources each mainloop kernel is compiled from (a recorded traffic figure
 # is valid only for the kernel source it was taken on)
 MAINLOOP_SOURCES = {
@@ -48,8 +49,8 @@ MAINLOOP_SOURCES = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default="long_fused")
     ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
@@ -224,7 +225,8 @@ def cpu_sample(cfg, inp, groups: int):
             "sample": f"full prepass of {len(heads)} heads + attention of {rows} query rows "
                       f"({len(gl)} 32-row groups x {len(heads)} heads) of {cfg.name}; "
                       f"extrapolated to all B*H heads and N rows",
-            "sample_seconds": round(t_pre + t_att, 2), "extrapolated_ms": total_s * 1e3}
+            "sample_seconds": round(t_pre + t_att, 2), "extrapolated_ms": total_s * 1e3,
+            "t_pre_s": t_pre, "t_att_per_group_s": t_att / len(gl)}
 
 
 def run_reference(args, cfg, rank, world):
@@ -232,12 +234,18 @@ def run_reference(args, cfg, rank, world):
         return
     import synth
     inp = synth.make_inputs(cfg, seed=0)
-    for _ in range(args.warmup):
+    # the first warm-up sample also sizes the timed ones: as many query groups
+    # per step as keep all the timed steps within REF_BUDGET_S
+    first = cpu_sample(cfg, inp, 1)
+    for _ in range(args.warmup - 1):
         cpu_sample(cfg, inp, 1)
+    per_step = REF_BUDGET_S / max(1, args.steps)
+    groups = int((per_step - first["t_pre_s"]) / max(first["t_att_per_group_s"], 1e-6))
+    groups = max(1, min(max(1, args.cpu_sample_groups // 2), groups))
     vals = []
     t_all = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(cpu_sample(cfg, inp, max(1, args.cpu_sample_groups // 2)))
+        vals.append(cpu_sample(cfg, inp, groups))
     wall = time.perf_counter() - t_all
     v = statistics.median(x["value"] for x in vals)
     ms = statistics.median(x["extrapolated_ms"] for x in vals)
@@ -409,7 +417,7 @@ def main():
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = {kk: vv for kk, vv in cpu_sample(cfg, inp, args.cpu_sample_groups).items()
-                                    if kk not in ("extrapolated_ms",)}
+                                    if kk not in ("extrapolated_ms", "t_pre_s", "t_att_per_group_s")}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--config", default="long_fused")
     ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-heads-per-chunk", type=int, default=4)
+    ap.add_argument("--e2e-one-stream", action="store_true", help="all chunks on one compute stream")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--cpu-sample-groups", type=int, default=16)
@@ -361,18 +363,20 @@ def main():
     value = whole_job_tops(cfg.ops, world, ms_step)
     ml_avg = statistics.mean(ml_ms)
 
-    # end to end through the public call with pinned host buffers
+    # end to end through the public call from pinned host buffers to a pinned
+    # host output: sage_attn_fwd_host copies each chunk of heads in, runs the
+    # path on it and copies its output back, overlapping the three
     host_out = torch.empty((B, N, H, D), dtype=torch.bfloat16).pin_memory()
-    ws_f = sage.workspace(sage.SAGE_OP_ATTN_FWD, B, N, H, D, dev)
-    h2d = sum(hb.numel() * 2 for hb in host_bufs)
+    hq, hk, hv = views(host_bufs)
+    hpc = min(H, args.e2e_heads_per_chunk)
+    ws_f = sage.workspace(sage.SAGE_OP_ATTN_FWD_HOST, B, N, hpc, D, dev)
+    h2d = sum(t.numel() * 2 for t in (hq, hk, hv))
     d2h = host_out.numel() * 2
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     def e2e_step():
-        for hb, db in zip(host_bufs, dev_bufs):
-            db.copy_(hb, non_blocking=True)
-        sage.sage_attn_fwd(q, k, v, out, 0.0, ws_f)
-        host_out.copy_(out, non_blocking=True)
+        sage.sage_attn_fwd_host(hq, hk, hv, q, k, v, host_out, out, 0.0, ws_f, hpc,
+                                two_streams=not args.e2e_one_stream)
 
     e2e_step()
     torch.cuda.synchronize()
@@ -411,7 +415,10 @@ def main():
                          "kernel": f"attn mainloop ({ml_name})",
                          "traffic": recorded_traffic(cfg.name, ml_name)},
             "e2e": {"value": whole_job_tops(cfg.ops, world, e2e_ms), "unit": UNIT,
-                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "call": f"sage_attn_fwd_host: chunks of 2, 2, then {hpc}, then 2 heads on "
+                            f"{'one compute stream' if args.e2e_one_stream else 'two compute streams'}, "
+                            "copies overlapped with compute"},
             "gpu_launches": args.steps * 8,  # seven prepass kernels and the mainloop
             "clocks": clk.summary(),
         }

@@ -31,6 +31,7 @@ SAGE_OP_ATTN_FWD = 2
 SAGE_OP_ATTN_FROM_QUANT = 3
 SAGE_OP_DEBUG_QK = 4
 SAGE_OP_QUANT_QKV = 5
+SAGE_OP_ATTN_FWD_HOST = 6
 
 SAGE_MAINLOOP_DEFAULT = 0
 SAGE_MAINLOOP_TCGEN05 = 1
@@ -44,7 +45,7 @@ EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_
            "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
            "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
-           "sage_attn_fwd_noalloc", "sage_debug_set_stall")
+           "sage_attn_fwd_noalloc", "sage_debug_set_stall", "sage_attn_fwd_host")
 SAGE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -94,6 +95,8 @@ def lib():
             "sage_debug_qk_s32": [P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
             "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
             "sage_debug_set_stall": [I, ctypes.c_longlong],
+            "sage_attn_fwd_host": [V, V, V, V, V, V, P, P, L64, L64, L64, I, I, I, I, ctypes.c_float, I, P, SZ,
+                                   P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -215,6 +218,59 @@ def sage_attn_fwd_noalloc(q, k, v, out, sm_scale, stream=None):
                                        out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
                                        _stream(stream)),
            "sage_attn_fwd_noalloc")
+
+
+def _host_view(t) -> sage_view_bf16:
+    import torch
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or t.stride(3) != 1 or t.is_cuda or not t.is_pinned():
+        raise ValueError("expected a pinned host bfloat16 [B, N, H, D] view with unit stride over D")
+    return sage_view_bf16(t.data_ptr(), t.stride(0), t.stride(1), t.stride(2))
+
+
+_aux = {}
+
+
+def _aux_streams(device):
+    """A second compute stream, two copy streams and three events per device,
+    created once; each event is recorded once here so that it exists before
+    its handle is passed on."""
+    import torch
+    key = torch.device(device).index
+    if key not in _aux:
+        with torch.cuda.device(key):
+            s_alt, s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+            evs = [torch.cuda.Event() for _ in range(3)]
+            for e in evs:
+                e.record()
+        _aux[key] = (s_alt, s_in, s_out, evs)
+    return _aux[key]
+
+
+def sage_attn_fwd_host(q_host, k_host, v_host, q_dev, k_dev, v_dev, out_host, out_dev, sm_scale, workspace,
+                       heads_per_chunk=4, stream=None, two_streams=True):
+    """sage_attn_fwd from pinned host tensors to a pinned host output, the
+    copies of each chunk of heads overlapped with the compute of the previous
+    one (see the header).  The device tensors receive the inputs and the
+    output; they must have the host tensors' strides.  The workspace is
+    workspace(SAGE_OP_ATTN_FWD_HOST, B, N, min(H, heads_per_chunk), D)."""
+    B, N, H, D = q_dev.shape
+    for t in (out_host, out_dev):
+        if t.stride(3) != 1 or tuple(t.shape) != (B, N, H, D):
+            raise ValueError("outputs must be [B, N, H, D] with unit stride over D")
+    if out_host.stride() != out_dev.stride():
+        raise ValueError("host and device outputs must have the same strides")
+    if out_dev.dtype != out_host.dtype or not out_dev.is_cuda or not out_host.is_pinned():
+        raise ValueError("out_dev must be a CUDA tensor and out_host a pinned host tensor of the same dtype")
+    s_alt, s_in, s_out, evs = _aux_streams(q_dev.device)
+    _check(lib().sage_attn_fwd_host(_host_view(q_host), _host_view(k_host), _host_view(v_host), _view(q_dev),
+                                    _view(k_dev), _view(v_dev), ctypes.c_void_p(out_host.data_ptr()), _ptr(out_dev),
+                                    out_dev.stride(0), out_dev.stride(1), out_dev.stride(2), B, N, H, D,
+                                    float(sm_scale), int(heads_per_chunk), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream),
+                                    ctypes.c_void_p(s_alt.cuda_stream if two_streams else None),
+                                    ctypes.c_void_p(s_in.cuda_stream), ctypes.c_void_p(s_out.cuda_stream),
+                                    *[ctypes.c_void_p(e.cuda_event) for e in evs]),
+           "sage_attn_fwd_host")
 
 
 def sage_read_device_status(workspace, stream=None) -> int:

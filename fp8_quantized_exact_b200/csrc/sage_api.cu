@@ -4,6 +4,9 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "sage_common.cuh"
 
 using namespace sage;
@@ -144,7 +147,7 @@ int resolved_mainloop() {
 
 AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const int8_t* k8,
                        const float* ks, const uint8_t* v8, const float* vs, void* out,
-                       int64_t osb, int64_t osn, int64_t osh, float sm_scale, void* ws) {
+                       int64_t osb, int64_t osn, int64_t osh, float sm_scale, void* status) {
   AttnParams p;
   p.q8 = q8; p.q_scale = qs; p.k8 = k8; p.k_scale = ks; p.v8 = v8; p.v_scale = vs;
   p.out = static_cast<uint16_t*>(out);
@@ -152,7 +155,7 @@ AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const i
   p.B = d.B; p.N = d.N; p.H = d.H; p.D = d.D;
   p.Nq = d.Nq; p.Nk = d.Nk; p.G32 = d.G32; p.T64 = d.T64;
   p.sl2 = log2_scale(sm_scale, d.D);
-  p.status = static_cast<DeviceStatus*>(ws);
+  p.status = static_cast<DeviceStatus*>(status);
   p.wait_limit = g_wait_limit;
   p.stall_tile = g_stall_tile;
   return p;
@@ -166,15 +169,106 @@ int run_mainloop(const AttnParams& p, cudaStream_t s) {
   }
 }
 
+
+// Copy the heads [h0, h1) of a [B, N, H, D] BF16 view between two buffers
+// laid out with the same element strides: per batch, one 2D copy whose rows
+// are the tokens when those heads are adjacent within a token's row, else
+// one 2D copy per head.
+int copy_heads(void* dst, const void* src, int64_t sb, int64_t sn, int64_t sh, int B, int N, int D,
+               int h0, int h1, cudaMemcpyKind kind, cudaStream_t s) {
+  const bool merged = sh == D && sn >= (int64_t)(h1 - h0) * D;
+  const int step = merged ? h1 - h0 : 1;
+  for (int b = 0; b < B; ++b)
+    for (int h = h0; h < h1; h += step) {
+      const size_t off = (size_t)((int64_t)b * sb + (int64_t)h * sh) * 2;
+      const size_t width = (size_t)step * D * 2;
+      const size_t pitch = N > 1 ? (size_t)sn * 2 : width;
+      if (cudaMemcpy2DAsync(static_cast<char*>(dst) + off, pitch, static_cast<const char*>(src) + off, pitch,
+                            width, (size_t)N, kind, s) != cudaSuccess)
+        return SAGE_ERR_CUDA;
+    }
+  return SAGE_OK;
+}
+
+// Pinned (page-locked or registered) host memory, and device-accessible memory.
+int pointer_type(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return (int)a.type;
+}
+bool host_pinned(const void* p) { return pointer_type(p) == (int)cudaMemoryTypeHost; }
+bool device_memory(const void* p) {
+  const int t = pointer_type(p);
+  return t == (int)cudaMemoryTypeDevice || t == (int)cudaMemoryTypeManaged;
+}
+
+// The path of sage_attn_fwd on checked arguments, its buffers carved from
+// `workspace`; device errors go to the status word at `status` (which the
+// callers clear).
+int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, void* out,
+             int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N, int H, int D,
+             float sm_scale, void* workspace, void* status, cudaStream_t s) {
+  int rc;
+  const Dims d = make_dims(B, N, H, D);
+  const Layout L = plan(SAGE_OP_ATTN_FWD, d);
+  int8_t* q8 = at<int8_t>(workspace, L.q8);
+  float* qs = at<float>(workspace, L.q_scale);
+  int8_t* k8 = at<int8_t>(workspace, L.k8);
+  float* ks = at<float>(workspace, L.k_scale);
+  float* km = at<float>(workspace, L.k_mean);
+  uint8_t* v8 = at<uint8_t>(workspace, L.v8);
+  float* vs = at<float>(workspace, L.v_scale);
+  // the separate prepass kernels: faster than the single-launch one (measured)
+  if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
+    return rc;
+  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_part),
+                             at<float>(workspace, L.v_amax), s)))
+    return rc;
+  return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
+                                  out_stride_h, sm_scale, status),
+                      s);
+}
+
+// Head counts of the chunks of sage_attn_fwd_host: 2, 2, then `hc` heads at
+// a time, and 2 at the end.  The first copy-in and the last copy-out overlap
+// nothing, so they are kept small; but not one head, whose rows (one head's
+// D elements per token) the copy engines move at half the rate of two heads'
+// (measured on B200: 26 against 52 GB/s for 256- and 512-byte rows).  Two
+// heads copy in faster than they compute, so the ramp never starves the
+// compute stream.
+std::vector<int> host_chunks(int H, int hc) {
+  std::vector<int> sizes;
+  const int tail = (H >= 6 && hc >= 2) ? 2 : 0;
+  int rem = H - tail;
+  for (int x : {2, 2}) {
+    if (rem <= 0) break;
+    const int c = std::min(std::min(x, hc), rem);
+    sizes.push_back(c);
+    rem -= c;
+  }
+  while (rem > 0) {
+    const int c = std::min(hc, rem);
+    sizes.push_back(c);
+    rem -= c;
+  }
+  if (tail) sizes.push_back(tail);
+  return sizes;
+}
 }  // namespace
 
 extern "C" {
 
 int sage_workspace_bytes(int op, int B, int N, int H, int D, size_t* bytes) {
-  if (!bytes || op < SAGE_OP_QUANT_QK || op > SAGE_OP_QUANT_QKV) return SAGE_ERR_INVALID_ARG;
+  if (!bytes || op < SAGE_OP_QUANT_QK || op > SAGE_OP_ATTN_FWD_HOST) return SAGE_ERR_INVALID_ARG;
   int rc = check_dims(B, N, H, D);
   if (rc) return rc;
-  *bytes = plan(op, make_dims(B, N, H, D)).total;
+  if (op == SAGE_OP_ATTN_FWD_HOST)  // two chunk workspaces of H heads
+    *bytes = 2 * align_up(plan(SAGE_OP_ATTN_FWD, make_dims(B, N, H, D)).total);
+  else
+    *bytes = plan(op, make_dims(B, N, H, D)).total;
   return SAGE_OK;
 }
 
@@ -299,27 +393,94 @@ int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* ou
   if (empty(B, N, H)) return SAGE_OK;
   if ((rc = check_view(q)) || (rc = check_view(k)) || (rc = check_view(v))) return rc;
   if ((rc = check_out(out, out_stride_b, out_stride_n, out_stride_h))) return rc;
-  const Dims d = make_dims(B, N, H, D);
-  const Layout L = plan(SAGE_OP_ATTN_FWD, d);
+  const Layout L = plan(SAGE_OP_ATTN_FWD, make_dims(B, N, H, D));
   if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
-  int8_t* q8 = at<int8_t>(workspace, L.q8);
-  float* qs = at<float>(workspace, L.q_scale);
-  int8_t* k8 = at<int8_t>(workspace, L.k8);
-  float* ks = at<float>(workspace, L.k_scale);
-  float* km = at<float>(workspace, L.k_mean);
-  uint8_t* v8 = at<uint8_t>(workspace, L.v8);
-  float* vs = at<float>(workspace, L.v_scale);
-  // the separate prepass kernels: faster than the single-launch one (measured)
-  if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
-    return rc;
-  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_part),
-                             at<float>(workspace, L.v_amax), s)))
-    return rc;
-  return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
-                                  out_stride_h, sm_scale, workspace),
-                      s);
+  return fwd_body(q, k, v, out, out_stride_b, out_stride_n, out_stride_h, B, N, H, D, sm_scale, workspace,
+                  workspace, s);
+}
+
+int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_bf16 v_host,
+                       sage_view_bf16 q_dev, sage_view_bf16 k_dev, sage_view_bf16 v_dev, void* out_host,
+                       void* out_dev, int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B,
+                       int N, int H, int D, float sm_scale, int heads_per_chunk, void* workspace,
+                       size_t workspace_bytes, void* stream, void* stream_alt, void* stream_in, void* stream_out,
+                       void* event_in, void* event_compute, void* event_out) {
+  int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return SAGE_OK;
+  if ((rc = check_view(q_dev)) || (rc = check_view(k_dev)) || (rc = check_view(v_dev))) return rc;
+  if ((rc = check_out(out_dev, out_stride_b, out_stride_n, out_stride_h))) return rc;
+  const sage_view_bf16* hv[3] = {&q_host, &k_host, &v_host};
+  const sage_view_bf16* dv[3] = {&q_dev, &k_dev, &v_dev};
+  for (int i = 0; i < 3; ++i) {
+    if (!hv[i]->data) return SAGE_ERR_INVALID_ARG;
+    if (hv[i]->stride_b != dv[i]->stride_b || hv[i]->stride_n != dv[i]->stride_n ||
+        hv[i]->stride_h != dv[i]->stride_h)
+      return SAGE_ERR_INVALID_ARG;
+    if (N > 1 && dv[i]->stride_n < D) return SAGE_ERR_UNSUPPORTED;
+  }
+  if (!out_host || !event_in || !event_compute || !event_out) return SAGE_ERR_INVALID_ARG;
+  if (N > 1 && out_stride_n < D) return SAGE_ERR_UNSUPPORTED;
+  const int hc = heads_per_chunk > 0 ? (heads_per_chunk < H ? heads_per_chunk : H) : (H < 4 ? H : 4);
+  // with a second compute stream the chunks alternate between two workspaces
+  const size_t per_chunk = align_up(plan(SAGE_OP_ATTN_FWD, make_dims(B, N, hc, D)).total);
+  const int n_ws = stream_alt ? 2 : 1;
+  if ((rc = check_ws(workspace, workspace_bytes, per_chunk * n_ws))) return rc;
+  for (int i = 0; i < 3; ++i)
+    if (!host_pinned(hv[i]->data) || !device_memory(dv[i]->data)) return SAGE_ERR_INVALID_ARG;
+  if (!host_pinned(out_host) || !device_memory(out_dev)) return SAGE_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t s_alt = static_cast<cudaStream_t>(stream_alt);
+  cudaStream_t s_in = static_cast<cudaStream_t>(stream_in);
+  cudaStream_t s_out = static_cast<cudaStream_t>(stream_out);
+  cudaEvent_t e_in = static_cast<cudaEvent_t>(event_in);
+  cudaEvent_t e_comp = static_cast<cudaEvent_t>(event_compute);
+  cudaEvent_t e_out = static_cast<cudaEvent_t>(event_out);
+  // Each cudaStreamWaitEvent below is enqueued before the next record of the
+  // same event, so it waits for the record just before it; three events serve
+  // every chunk.
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  if ((rc = clear_status(workspace, s))) return rc;
+  // the caller's earlier work on `stream` (users of the device buffers) first
+  if (!ok(cudaEventRecord(e_in, s)) || !ok(cudaStreamWaitEvent(s_in, e_in, 0)) ||
+      !ok(cudaStreamWaitEvent(s_out, e_in, 0)) || (s_alt && !ok(cudaStreamWaitEvent(s_alt, e_in, 0))))
+    return SAGE_ERR_CUDA;
+  const std::vector<int> chunks = host_chunks(H, hc);
+  int h0 = 0;
+  for (size_t j = 0; j < chunks.size(); h0 += chunks[j], ++j) {
+    const int h1 = h0 + chunks[j];
+    // even chunks on `stream` with the first workspace, odd ones on the
+    // second stream with the second: a chunk's start overlaps the last wave
+    // of the chunk before
+    const bool alt = s_alt && (j & 1);
+    cudaStream_t sc = alt ? s_alt : s;
+    void* wsc = static_cast<char*>(workspace) + (alt ? per_chunk : 0);
+    for (int i = 0; i < 3; ++i)
+      if ((rc = copy_heads(const_cast<void*>(dv[i]->data), hv[i]->data, dv[i]->stride_b, dv[i]->stride_n,
+                           dv[i]->stride_h, B, N, D, h0, h1, cudaMemcpyHostToDevice, s_in)))
+        return rc;
+    if (!ok(cudaEventRecord(e_in, s_in)) || !ok(cudaStreamWaitEvent(sc, e_in, 0))) return SAGE_ERR_CUDA;
+    sage_view_bf16 cv[3];
+    for (int i = 0; i < 3; ++i) {
+      cv[i] = *dv[i];
+      cv[i].data = static_cast<const uint16_t*>(dv[i]->data) + (int64_t)h0 * dv[i]->stride_h;
+    }
+    void* co = static_cast<uint16_t*>(out_dev) + (int64_t)h0 * out_stride_h;
+    if ((rc = fwd_body(cv[0], cv[1], cv[2], co, out_stride_b, out_stride_n, out_stride_h, B, N, h1 - h0, D,
+                       sm_scale, wsc, workspace, sc)))
+      return rc;
+    if (!ok(cudaEventRecord(e_comp, sc)) || !ok(cudaStreamWaitEvent(s_out, e_comp, 0))) return SAGE_ERR_CUDA;
+    if ((rc = copy_heads(out_host, out_dev, out_stride_b, out_stride_n, out_stride_h, B, N, D, h0, h1,
+                         cudaMemcpyDeviceToHost, s_out)))
+      return rc;
+  }
+  // the caller's stream completes after the last copy-out, which follows every
+  // chunk's compute (each copy-out waited for its chunk)
+  if (!ok(cudaEventRecord(e_out, s_out)) || !ok(cudaStreamWaitEvent(s, e_out, 0))) return SAGE_ERR_CUDA;
+  return SAGE_OK;
 }
 
 int sage_read_device_status(const void* workspace, void* stream) {

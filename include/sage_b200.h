@@ -84,7 +84,9 @@ enum sage_op {
   SAGE_OP_ATTN_FWD = 2,
   SAGE_OP_ATTN_FROM_QUANT = 3,
   SAGE_OP_DEBUG_QK = 4,
-  SAGE_OP_QUANT_QKV = 5
+  SAGE_OP_QUANT_QKV = 5,
+  SAGE_OP_ATTN_FWD_HOST = 6  /* sage_attn_fwd_host with chunks of H heads and
+                                two compute streams (two chunk workspaces) */
 };
 
 /* Mainloop implementations.  DEFAULT, TCGEN05 and MMA_SYNC compute the
@@ -191,6 +193,55 @@ SAGE_API int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v,
                   int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N,
                   int H, int D, float sm_scale, void* workspace, size_t workspace_bytes,
                   void* stream);
+
+/* sage_attn_fwd from and to host memory, with the copies overlapped with the
+ * computation (no counterpart in the pages: a packaging of the same path for
+ * callers whose tensors live on the host).  Every (b, h) head is independent
+ * (per-head K mean and V scale; "Sage2 Blackwell Mainloop", section
+ * "Decision"), so the heads are processed in chunks: chunk j's Q/K/V heads
+ * are copied host -> device on `stream_in`, the path of sage_attn_fwd runs on
+ * them on a compute stream, and their output is copied device -> host on
+ * `stream_out`; the copy-in of chunk j+1 and the copy-out of chunk j-1
+ * overlap the compute of chunk j.  The chunks hold 2, 2 heads, then
+ * `heads_per_chunk` (<= 0 selects 4) at a time, and 2 at the end, so that
+ * the first copy-in and the last copy-out, which overlap nothing, are small
+ * (not one head: the copy engines move one head's 256-byte rows at half the
+ * rate of wider ones).  With `stream_alt` non-NULL the chunks alternate between
+ * `stream` and `stream_alt` (each with its own half of the workspace), so
+ * that a chunk's first launches fill the SMs that the previous chunk's last
+ * wave leaves idle.  The bytes written are those of sage_attn_fwd on the
+ * whole problem.
+ *   q_host, k_host, v_host  host views ([B, N, H, D] BF16, unit stride over
+ *                           d) in pinned memory (cudaHostAlloc or
+ *                           cudaHostRegister); they may alias one buffer.
+ *   q_dev, k_dev, v_dev     device views with the same strides, which
+ *                           receive the inputs (aliasing as the host views
+ *                           do); each needs stride_n >= D when N > 1.
+ *   out_host, out_dev       BF16 [B, N, H, D] outputs with the strides
+ *                           out_stride_* (pinned host memory; device memory).
+ *   workspace               sage_workspace_bytes(SAGE_OP_ATTN_FWD_HOST, B,
+ *                           N, min(H, heads_per_chunk), D) bytes (half of
+ *                           that suffices without `stream_alt`), 256-byte
+ *                           aligned; its status word covers all chunks.
+ *   stream, stream_alt,     streams of the current device (`stream` is the
+ *   stream_in, stream_out   caller's: the call starts after its earlier work
+ *                           and its later work starts after the last
+ *                           copy-out; `stream_alt` may be NULL).
+ *   event_in, event_compute,
+ *   event_out               three events created by the caller (timing
+ *                           disabled is best), recorded and waited on in
+ *                           turn; they must not be in use elsewhere until
+ *                           `stream` has passed this call.
+ * Returns SAGE_ERR_INVALID_ARG when a host buffer is not pinned or a device
+ * buffer is not device memory, or when host and device strides differ;
+ * otherwise as sage_attn_fwd.  Everything is enqueued asynchronously; the
+ * host output is complete once `stream` has completed the call. */
+SAGE_API int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_bf16 v_host,
+                       sage_view_bf16 q_dev, sage_view_bf16 k_dev, sage_view_bf16 v_dev, void* out_host,
+                       void* out_dev, int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B,
+                       int N, int H, int D, float sm_scale, int heads_per_chunk, void* workspace,
+                       size_t workspace_bytes, void* stream, void* stream_alt, void* stream_in, void* stream_out,
+                       void* event_in, void* event_compute, void* event_out);
 
 /* Where the quantised tensors of sage_attn_fwd live inside its workspace
  * (byte offsets from the workspace base, layouts above). */

@@ -49,6 +49,9 @@ def test_workspace_sizes(lib):
     offs = [lay[k] for k in ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean", "v_fp8", "v_scale")]
     assert offs == sorted(offs) and all(o % 1024 == 0 for o in offs) and offs[0] >= 256
     assert lay["total"] == sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD, 1, 1000, 8, 128)
+    # the host pipeline: two chunk workspaces, each rounded up to 1024 bytes
+    one = sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD, 1, 1000, 4, 128)
+    assert sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD_HOST, 1, 1000, 4, 128) == 2 * ((one + 1023) // 1024 * 1024)
 
 
 def test_argument_errors_need_no_device(lib):
@@ -101,6 +104,25 @@ def test_argument_errors_need_no_device(lib):
         assert lib.sage_get_mainloop() == which
     assert lib.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT) == sage.SAGE_OK
     assert lib.sage_debug_qk_s32(4096, 4096, 1, 100, 2, 64, 0, 2, 0, 0, 4096, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
+    host = lib.sage_attn_fwd_host
+    other = sage.sage_view_bf16(8192, 256 * 2 * 128, 2 * 128, 128)
+    narrow = sage.sage_view_bf16(4096, 256 * 2 * 128, 32, 128)
+
+    def fh(qh=good, qd=good, out_host=4096, D=128, hpc=4, ws_bytes=1 << 24, ev=4096, N=10):
+        # (q/k/v host, q/k/v dev, out host, out dev, out strides, B, N, H, D, sm_scale, heads_per_chunk,
+        #  ws, ws bytes, stream, stream_in, stream_out, three events)
+        return host(qh, good, good, qd, good, good, out_host, 4096, 0, 256, 128, 1, N, 2, D, 0.0, hpc, 4096,
+                    ws_bytes, None, None, None, None, ev, ev, ev)
+    assert fh(D=96) == sage.SAGE_ERR_UNSUPPORTED
+    assert fh(qd=odd) == sage.SAGE_ERR_UNSUPPORTED
+    assert fh(qh=null) == sage.SAGE_ERR_INVALID_ARG
+    assert fh(qh=other) == sage.SAGE_ERR_INVALID_ARG          # host and device strides differ
+    assert fh(out_host=None) == sage.SAGE_ERR_INVALID_ARG
+    assert fh(ev=None) == sage.SAGE_ERR_INVALID_ARG
+    assert fh(ws_bytes=100) == sage.SAGE_ERR_WORKSPACE
+    assert host(narrow, good, good, narrow, good, good, 4096, 4096, 0, 256, 128, 1, 10, 2, 64, 0.0, 4, 4096,
+                1 << 24, None, None, None, None, 4096, 4096, 4096) == sage.SAGE_ERR_UNSUPPORTED  # stride_n < D
+    assert fh(N=0) == sage.SAGE_OK
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

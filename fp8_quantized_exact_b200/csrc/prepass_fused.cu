@@ -226,6 +226,7 @@ __device__ bool wait_head(const FusedArgs& a, int bh) {
 }
 
 // K: 128 threads per 64-row chunk, two chunks at a time; x' = fl32(x - km).
+// The raw BF16 chunks stay in registers between the amax and code passes.
 template <int D>
 __device__ void k_quant(const FusedArgs& a, int bh, int c0, int c1) {
   constexpr int SEG = D / 8;
@@ -241,22 +242,22 @@ __device__ void k_quant(const FusedArgs& a, int bh, int c0, int c1) {
   for (int cb = c0; cb < c1; cb += 2) {
     const int chunk = cb + half;
     const bool live = chunk < c1;
-    float xs[PER][8];
+    uint4 xr[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int row = chunk * kKTile + (t + 128 * i) / SEG;
+      xr[i] = live && row < a.N ? ld16(a.k + b * a.ksb + (int64_t)row * a.ksn + h * a.ksh + col)
+                                : make_uint4(0, 0, 0, 0);
+    }
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int row = chunk * kKTile + (t + 128 * i) / SEG;
       if (live && row < a.N) {
         float f[8];
-        unpack8(ld16(a.k + b * a.ksb + (int64_t)row * a.ksn + h * a.ksh + col), f);
+        unpack8(xr[i], f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          xs[i][j] = __fsub_rn(f[j], km[j]);
-          amax = fmaxf(amax, fabsf(xs[i][j]));
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xs[i][j] = 0.0f;
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fsub_rn(f[j], km[j])));
       }
     }
     amax = warp_max(amax);
@@ -270,56 +271,84 @@ __device__ void k_quant(const FusedArgs& a, int bh, int c0, int c1) {
       int8_t* dst = a.k8 + ((size_t)bh * a.Nk + (size_t)chunk * kKTile) * D;
 #pragma unroll
       for (int i = 0; i < PER; ++i) {
-        const int row = (t + 128 * i) / SEG;
-        uint2 o;
-        o.x = code_i8(xs[i][0], inv) | code_i8(xs[i][1], inv) << 8 | code_i8(xs[i][2], inv) << 16 |
-              code_i8(xs[i][3], inv) << 24;
-        o.y = code_i8(xs[i][4], inv) | code_i8(xs[i][5], inv) << 8 | code_i8(xs[i][6], inv) << 16 |
-              code_i8(xs[i][7], inv) << 24;
-        *reinterpret_cast<uint2*>(dst + (size_t)row * D + col) = o;
+        const int r = (t + 128 * i) / SEG;
+        uint2 o = make_uint2(0u, 0u);  // pad rows get zero codes
+        if (chunk * kKTile + r < a.N) {
+          float f[8], x[8];
+          unpack8(xr[i], f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) x[j] = __fsub_rn(f[j], km[j]);
+          o.x = code_i8(x[0], inv) | code_i8(x[1], inv) << 8 | code_i8(x[2], inv) << 16 | code_i8(x[3], inv) << 24;
+          o.y = code_i8(x[4], inv) | code_i8(x[5], inv) << 8 | code_i8(x[6], inv) << 16 | code_i8(x[7], inv) << 24;
+        }
+        *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
       }
     }
   }
 }
 
-// V: D/2 threads per 64-token chunk (two channels each), 512/D chunks at a
-// time; bytes transposed in registers, 64 bytes per channel row.
+// V: 128 tokens at a time staged in shared memory with 16-byte loads (the
+// chunk index of a row XORed with bits 4-5 of its token, so that the column
+// reads hit distinct banks); each thread then converts 16 consecutive tokens
+// of one channel to E4M3 (token t in byte t of the channel's row) and writes
+// them as one 16-byte vector.
+constexpr int kVBlock = 2 * kKTile;
+
 template <int D>
 __device__ void v_quant(const FusedArgs& a, int bh, int c0, int c1) {
-  constexpr int TPCH = D / 2, CH_AT = kThreadsP / TPCH;
+  constexpr int SEG = D / 8;
+  constexpr int LOADS = kVBlock * SEG / kThreadsP;
+  constexpr int RUNS = D * (kVBlock / 16) / kThreadsP;
+  __shared__ __align__(16) uint4 tile[kVBlock * SEG];
   const int b = bh / a.H, h = bh % a.H;
-  const int d0 = (threadIdx.x % TPCH) * 2;
-  const float a0 = __ldcg(a.v_amax + (size_t)bh * D + d0);
-  const float a1 = __ldcg(a.v_amax + (size_t)bh * D + d0 + 1);
-  const float inv0 = a0 > 0.0f ? __fdiv_rn(448.0f, a0) : 0.0f;
-  const float inv1 = a1 > 0.0f ? __fdiv_rn(448.0f, a1) : 0.0f;
-  const uint16_t* vp = a.v + b * a.vsb + h * a.vsh + d0;
+  const uint16_t* vp = a.v + b * a.vsb + h * a.vsh;
+  const float* am = a.v_amax + (size_t)bh * D;
+  const uint16_t* ts = reinterpret_cast<const uint16_t*>(tile);
+  const int tok1 = min(c1 * kKTile, a.Nk);  // end of this item's tokens (padded length)
 #pragma unroll 1
-  for (int cb = c0; cb < c1; cb += CH_AT) {
-    const int c = cb + threadIdx.x / TPCH;
-    if (c >= c1) continue;
-    uint32_t w0[16], w1[16];
+  for (int n0 = c0 * kKTile; n0 < tok1; n0 += kVBlock) {
+    __syncthreads();  // the previous block's column reads are done
+    // staged in two rounds of loads, to stay within the registers
 #pragma unroll
-    for (int i = 0; i < 16; ++i) { w0[i] = 0u; w1[i] = 0u; }
+    for (int i0 = 0; i0 < LOADS; i0 += LOADS / 2) {
+      uint4 x[LOADS / 2];
 #pragma unroll
-    for (int t = 0; t < kKTile; ++t) {
-      const int n = c * kKTile + t;
-      if (n < a.N) {
-        const uint32_t pair = __ldg(reinterpret_cast<const uint32_t*>(vp + (int64_t)n * a.vsn));
-        const float x0 = __uint_as_float(pair << 16), x1 = __uint_as_float(pair & 0xFFFF0000u);
-        const uint16_t e = e4m3x2(__fmul_rn(x0, inv0), __fmul_rn(x1, inv1));
-        const uint32_t b0 = a0 > 0.0f ? (e & 0xFFu) : 0u;
-        const uint32_t b1 = a1 > 0.0f ? (e >> 8) : 0u;
-        w0[t >> 2] |= b0 << (8 * (t & 3));
-        w1[t >> 2] |= b1 << (8 * (t & 3));
+      for (int i = 0; i < LOADS / 2; ++i) {
+        const int idx = threadIdx.x + kThreadsP * (i0 + i);
+        const int r = idx / SEG, k = idx % SEG;
+        x[i] = n0 + r < a.N ? ld16(vp + (int64_t)(n0 + r) * a.vsn + k * 8) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < LOADS / 2; ++i) {
+        const int idx = threadIdx.x + kThreadsP * (i0 + i);
+        const int r = idx / SEG, k = idx % SEG;
+        tile[r * SEG + (k ^ ((r >> 4) & 3))] = x[i];
       }
     }
-    uint8_t* r0 = a.v8 + ((size_t)bh * D + d0) * a.Nk + (size_t)c * kKTile;
-    uint8_t* r1 = r0 + a.Nk;
+    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      reinterpret_cast<uint4*>(r0)[i] = make_uint4(w0[4 * i], w0[4 * i + 1], w0[4 * i + 2], w0[4 * i + 3]);
-      reinterpret_cast<uint4*>(r1)[i] = make_uint4(w1[4 * i], w1[4 * i + 1], w1[4 * i + 2], w1[4 * i + 3]);
+    for (int i = 0; i < RUNS; ++i) {
+      const int idx = threadIdx.x + kThreadsP * i;
+      const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
+      const int cb = rest % SEG, hf = rest / SEG;
+      const int t0 = hf * kKTile + 16 * q;
+      if (n0 + hf * kKTile >= tok1) continue;
+      const int ch = cb * 8 + cl;
+      const float amx = __ldcg(am + ch);
+      const float inv = amx > 0.0f ? __fdiv_rn(448.0f, amx) : 0.0f;
+      const uint16_t* col = ts + (cb ^ q) * 8 + cl;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = t0 + 4 * j;
+        const uint32_t lo = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[t * D]), inv),
+                                   __fmul_rn(bf16_bits_to_f32(col[(t + 1) * D]), inv));
+        const uint32_t hi = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[(t + 2) * D]), inv),
+                                   __fmul_rn(bf16_bits_to_f32(col[(t + 3) * D]), inv));
+        w[j] = amx > 0.0f ? (lo | (hi << 16)) : 0u;
+      }
+      uint8_t* dst = a.v8 + ((size_t)bh * D + ch) * a.Nk + n0 + t0;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }

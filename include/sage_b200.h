@@ -162,8 +162,8 @@ SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t*
  * "Completed P1 And P2").  A persistent kernel takes work in head-major
  * order; the K/V quantisation of a head waits, bounded, for the head's
  * statistics (a wait that runs out leaves SAGE_ERR_TIMEOUT in the status
- * word).  On one B200 it is slower than the two separate calls (1.75 ms
- * against 1.21 ms at B1 N37810 H56 D128), which keep more memory streams in
+ * word).  On one B200 it is slower than the two separate calls (0.91 ms
+ * against 0.75 ms at B1 N37810 H56 D128), which keep more memory streams in
  * flight; sage_attn_fwd uses the separate kernels.
  * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QKV, ...), 256-byte
  * aligned; concurrent calls need separate workspaces. */

@@ -9,25 +9,23 @@
  * does.  It shares no code with the CUDA library.
  *
  * Sources (the research pages this method is described on):
- *  - "Sage2 Blackwell Mainloop" (SAGE2_BLACKWELL_DESIGN.md), section
- *    "Existing Contract": projection-strided BF16 NHD input, per-warp INT8 Q
- *    in 128-row blocks of 32-row warp groups, per-block INT8 K with 64-row
- *    blocks, FP8 V with a per-channel scale, fp32+fp16 instantaneous-buffer
- *    accumulation, contiguous BF16 NHD output.
- *  - "State-Ownership Architecture Decision" (vortex_exact_attention
- *    DESIGN.md), section "Non-Negotiable Dataflow": exact global K mean and
- *    V scale prepasses; all K64/V64 tiles in increasing order; per tile QK,
+ *  - "Sage2 Blackwell Mainloop", section "Existing Contract":
+ *    projection-strided BF16 NHD input, per-warp INT8 Q in 128-row blocks of
+ *    32-row warp groups, per-block INT8 K with 64-row blocks, FP8 V with a
+ *    per-channel scale, fp32+fp16 instantaneous-buffer accumulation,
+ *    contiguous BF16 NHD output.
+ *  - "State-Ownership Architecture Decision", section "Non-Negotiable
+ *    Dataflow": exact global K mean and V scale prepasses; all K64/V64 tiles
+ *    in increasing order; per tile QK,
  *    score scaling, max update, denominator update, FP8 probability
  *    conversion, two K32 FP16 PV MMAs and the FP32 RO addition; and the
  *    "exact handoff record" paragraph: ro_rescale (the old-max rescale) is
  *    applied before the tile's PV, and the final normalisation uses the FP32
  *    reciprocal of d, then the V scale, then BF16 conversion.
- *  - "Sage2 SM89 Temporal Pair Experiment" (research/sage2_temporal_pair),
- *    section "Candidate": the per-tile order
- *    QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV.
+ *  - "Sage2 SM89 Temporal Pair Experiment", section "Candidate": the
+ *    per-tile order QK -> update_mdo -> accumulate_d -> RS_32_to_8 -> PV.
  *
- * Readings taken where the pages are silent (each is also listed in the
- * design notes):
+ * Readings taken where the pages are silent:
  *  R1 K mean: per (b,h,d) an FP64 sum over tokens, sequential inside each
  *     64-token chunk, then the chunk partials added sequentially in chunk
  *     order; km = float(sum / N), one round-to-nearest-even.

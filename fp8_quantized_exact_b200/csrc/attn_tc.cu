@@ -83,7 +83,7 @@ struct TcSmem {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], r_free[2];
-  uint64_t o_full[2], o_free[2];
+  uint64_t o_full[2], o_free;  // o_free: both FP16 buffers of a tile have been read
   uint64_t m_full[4][2];
   uint64_t fin, done;
   uint64_t drain_qk, drain_pv;
@@ -123,9 +123,9 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       mbar_init(&sm.p_full[i], kQTile);
       mbar_init(&sm.r_free[i], 2 * kQTile + 1);  // output owners and the PV issuer
       mbar_init(&sm.o_full[i], 1);
-      mbar_init(&sm.o_free[i], 2 * kQTile);
       for (int q = 0; q < 4; ++q) mbar_init(&sm.m_full[q][i], 32);
     }
+    mbar_init(&sm.o_free, 2 * kQTile);
     mbar_init(&sm.fin, 2 * kQTile);
     mbar_init(&sm.done, kQTile);
     mbar_init(&sm.drain_qk, 1);
@@ -248,16 +248,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
           break;
         }
         tc_fence_after();
-        // 32 columns at a time (16 registers of FP16 pairs); the buffer is
-        // released once the last columns are in registers
+        // 32 columns at a time (16 registers of FP16 pairs); both buffers are
+        // released once the last columns of slice 1 are in registers (slice
+        // 0 was read before, so one arrival per tile covers both)
 #pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 32) {
           uint32_t hv[16];
           tmem_ld16_pack16(lane_addr + kColO + 128 * sl + c_base + c0, hv);
           tmem_wait_ld();
-          if (c0 + 32 >= DH) {
+          if (sl == 1 && c0 + 32 >= DH) {
             tc_fence_before();
-            mbar_arrive(&sm.o_free[sl]);  // the buffer may be overwritten now
+            mbar_arrive(&sm.o_free);  // both buffers may be overwritten now
           }
           // RO += float(tmp), one rounding per element (float(tmp) is exact):
           // one mixed-precision add (FP16 operand, FP32 accumulator) each
@@ -356,12 +357,12 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       const int g = t >> 1, sb = g & 1, st = g % kStages, half = t & 1;
       // this tile's probabilities; the V^T stage, which arrived with the K stage
       // the QK issuer waited for; both FP16 buffers read by the output owners
+      // (one wait: a single wake-up of this warp per tile)
       const bool ok =
           wait_bounded(&sm.p_full[half], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 12, p.wait_limit) &&
           (half == 1 ||
            wait_bounded(&sm.kv_full[st], (uint32_t)((g / kStages) & 1), abort_flag, p.status, 18, p.wait_limit)) &&
-          wait_bounded(&sm.o_free[0], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit) &&
-          wait_bounded(&sm.o_free[1], (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit);
+          wait_bounded(&sm.o_free, (uint32_t)((t & 1) ^ 1), abort_flag, p.status, 13, p.wait_limit);
       __syncwarp();  // every lane has seen the phases before lane 0 acts on them
       if (!ok) break;
       tc_fence_after();

@@ -229,6 +229,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
+      // slice 0 first: its MMA was issued after this tile's probabilities were
+      // in, so p_full(t) is complete by then and its wait below is one test
+      // (one wake-up of this warp per tile)
+      if (!wait_bounded(&sm.o_full[0], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) break;
       if (!wait_bounded(&sm.p_full[bi], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 3, p.wait_limit)) break;
       const float r = sm.r_ring[bi][i];
       mbar_arrive(&sm.r_free[bi]);
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       }
 #pragma unroll
       for (int sl = 0; sl < 2; ++sl) {  // K32 slice sl of tile t sits in buffer sl
-        if (!wait_bounded(&sm.o_full[sl], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
+        if (sl == 1 && !wait_bounded(&sm.o_full[1], (uint32_t)(t & 1), abort_flag, p.status, 4, p.wait_limit)) {
           ok = false;
           break;
         }

@@ -42,3 +42,37 @@ def test_withheld_tile_times_out_and_context_survives():
     out2, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05)
     qz = oracle.quantize(inp.q, inp.k, inp.v)
     gu.compare_out(out2.float().cpu().numpy(), oracle.bf16_bits_to_float(oracle.attention(qz)), "after timeout")
+
+
+def test_timeout_inside_the_host_pipeline_reaches_its_status_word():
+    # a withheld tile in every chunk of sage_attn_fwd_host (chunks on both
+    # compute streams): the one status word of its workspace reports the
+    # timeout, and the next call gives the bytes of sage_attn_fwd
+    import fp8_quantized_exact_b200 as sage
+    from fp8_quantized_exact_b200 import build
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    build.build()
+    dev = torch.device("cuda:0")
+    sage.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT)
+    if sage.sage_get_mainloop() != sage.SAGE_MAINLOOP_TCGEN05:
+        pytest.skip("the bounded waits live in the tcgen05 mainloop")
+    inp = synth.custom(1, 700, 8, 128, seed=7)
+    host = [torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).pin_memory()
+            for a in (inp.q, inp.k, inp.v)]
+    (q, k, v), _ = gu.to_device(inp, dev)
+    B, N, H, D = q.shape
+    out_d = torch.empty_like(q)
+    out_h = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    ws = sage.workspace(sage.SAGE_OP_ATTN_FWD_HOST, B, N, 2, D, dev)
+    try:
+        sage.sage_debug_set_stall(3, 2_000_000)
+        sage.sage_attn_fwd_host(*host, q, k, v, out_h, out_d, 0.0, ws, 2)
+        st = sage.sage_read_device_status(ws)
+    finally:
+        sage.sage_debug_set_stall(-1, 0)
+    assert st == sage.SAGE_ERR_TIMEOUT, sage.sage_strerror(st)
+    sage.sage_attn_fwd_host(*host, q, k, v, out_h, out_d, 0.0, ws, 2)
+    assert sage.sage_read_device_status(ws) == sage.SAGE_OK
+    ref, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05)
+    assert torch.equal(out_h.view(torch.int16), ref.cpu().view(torch.int16))

@@ -23,7 +23,8 @@ def declared_functions():
     names = set()
     for fn in os.listdir(os.path.join(ROOT, "include")):
         if fn.endswith(".h"):
-            text = open(os.path.join(ROOT, "include", fn)).read()
+            with open(os.path.join(ROOT, "include", fn)) as f:
+                text = f.read()
             names |= set(re.findall(r"SAGE_API\s+[\w\s\*]+?\b(sage_\w+)\s*\(", text))
     return names
 

@@ -214,15 +214,16 @@ __global__ void __launch_bounds__(kThreadsF, 1)
     bool ok = true;
     for (int t = 0; t < T && ok; ++t) {
       const int bi = t & 1;
-      // PV(t - 1) has completed, so the accumulator holds tiles 0 .. t-1.  The
-      // parity is unambiguous: this warp saw tile t - 5 complete on the same
+      // this tile's probabilities first (the wait that usually sleeps), then
+      // PV(t - 1), after which the accumulator holds tiles 0 .. t-1.  The
+      // o_acc parity is unambiguous: this warp saw tile t - 5 complete on the same
       // barrier, and the next MMAs that complete it, PV(t + 3), need the
       // probabilities of tile t + 3, which wait for this warp's r_free
       // arrival for tile t + 1.
+      if (!wait_bounded(&sm.p_full[bi], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 3, p.wait_limit)) break;
       if (t > 0 && !wait_bounded(&sm.o_acc[(t - 1) & 3], (uint32_t)(((t - 1) >> 2) & 1), abort_flag, p.status, 20,
                                  p.wait_limit))
         break;
-      if (!wait_bounded(&sm.p_full[bi], (uint32_t)((t >> 1) & 1), abort_flag, p.status, 3, p.wait_limit)) break;
       // r and the flags are read before the arrival: after it the softmax
       // owners of tile t + 2 may overwrite them
       const float r = sm.r_ring[bi][i];

@@ -25,9 +25,12 @@
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers on the current CUDA device and
- *     are owned by the caller.  The library allocates nothing, frees nothing
- *     and does not synchronise (except sage_read_device_status).  Work is
- *     enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     are owned by the caller, except the pinned host buffers that
+ *     sage_attn_fwd_host copies from and to.  The library allocates nothing,
+ *     frees nothing and does not synchronise the host (except
+ *     sage_read_device_status).  Work is enqueued on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream), and on the further
+ *     streams the caller passes to sage_attn_fwd_host.
  *   - Shapes: B (batch), N (tokens), H (heads), D (head dim, 64 or 128).
  *     B, N or H equal to 0 is an empty problem: SAGE_OK, nothing launched.
  *   - BF16 views carry element strides (b, n, h); d has unit stride.  The

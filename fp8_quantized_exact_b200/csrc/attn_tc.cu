@@ -13,14 +13,17 @@
 //               probabilities, its part of the denominator, and writes the
 //               E4M3 probabilities back to TMEM over the scores.
 //   warps 8-15  output owners: thread (w, lane) owns half of the FP32 output
-//               row RO of row 32*(w%4)+lane in registers.  Per tile it applies
-//               r, then adds each FP16 K32 buffer (read from TMEM) in order;
-//               at the end it applies 1/d and the V scale and stores BF16.
+//               row RO of row 32*(w%4)+lane in registers.  Per tile it waits
+//               for the first FP16 K32 buffer, reads r, applies it, then adds
+//               each buffer (read from TMEM) in order, releasing both with
+//               one arrival once the second is in registers; at the end it
+//               applies 1/d and the V scale and stores BF16.
 //   warp 16     TMA producer: the Q tile once, then K and V^T stages of 128
 //               keys (two tiles) into a ring of shared-memory stages.
 //   warp 17     QK issuer: per 128-key group four INT8 MMAs (N = 128, K = 32
 //               each) into one of two TMEM score buffers.
-//   warp 18     PV issuer: once a tile's probabilities are in,
+//   warp 18     PV issuer: once a tile's probabilities are in and both FP16
+//               buffers of the previous tile have been read (one barrier),
 //               per K32 slice one E4M3 MMA, with the probabilities as the TMEM
 //               A operand, into an FP16 accumulator that starts at zero (the
 //               instantaneous buffer), one TMEM buffer per slice.

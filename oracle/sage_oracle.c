@@ -172,7 +172,11 @@ static float f16_to_f32(uint16_t h) {
 
 /* round-half-even to integer, then clamp to the INT8 code range */
 static int8_t quant_i8(float prod) {
+#if ORACLE_PLANT == 14
+  float r = roundf(prod); /* planted: ties away from zero */
+#else
   float r = nearbyintf(prod);
+#endif
   if (r > 127.0f) r = 127.0f;
   if (r < -127.0f) r = -127.0f;
   return (int8_t)r;
@@ -210,6 +214,9 @@ int oracle_k_mean(const uint16_t* k, int64_t sb, int64_t sn, int64_t sh,
         }
 #if ORACLE_PLANT == 1
         km[((int64_t)b * H + h) * D + d] = 0.0f; /* planted: smoothing dropped */
+#elif ORACLE_PLANT == 15
+        km[((int64_t)b * H + h) * D + d] =      /* planted: mean over the padded length */
+            N > 0 ? (float)(total / (double)(64 * ((N + 63) / 64))) : 0.0f;
 #else
         km[((int64_t)b * H + h) * D + d] = N > 0 ? (float)(total / (double)N) : 0.0f;
 #endif
@@ -387,7 +394,11 @@ int oracle_attn_rows(const int8_t* q8, const float* q_scale, const int8_t* k8, c
 
   for (int ri = 0; ri < rows; ++ri) {
     const int i = row0 + ri;
+#if ORACLE_PLANT == 16
+    const float qs = q_scale[bh * ng + i / 64]; /* planted: Q scale read per 64 rows */
+#else
     const float qs = q_scale[bh * ng + i / 32];
+#endif
     float m = -INFINITY, dsum = 0.0f;
     for (int e = 0; e < D; ++e) RO[e] = 0.0f;
 
@@ -400,7 +411,11 @@ int oracle_attn_rows(const int8_t* q8, const float* q_scale, const int8_t* k8, c
       float tmax = -INFINITY;
       for (int jj = 0; jj < 64; ++jj) {
         int j = j0 + jj;
+#if ORACLE_PLANT == 13
+        if (j >= j1) { s[jj] = 0.0f; continue; }       /* planted: tail keys not masked */
+#else
         if (j >= j1) { s[jj] = -INFINITY; continue; }  /* tail mask */
+#endif
         int32_t S = 0;
 #if ORACLE_PLANT == 5
         for (int e = 0; e < D; ++e) S += (int32_t)Q[(int64_t)i * D + e] * K[(int64_t)j * D + (D - 1 - e)];
@@ -426,20 +441,33 @@ int oracle_attn_rows(const int8_t* q8, const float* q_scale, const int8_t* k8, c
 #else
         p[jj] = (float)exp2((double)(s[jj] - m_new));
 #endif
+#if ORACLE_PLANT == 10
+        rowsum = rowsum + (float)e4m3_decode(e4m3_encode(p[jj])); /* planted: d from E4M3 p */
+#else
         rowsum = rowsum + p[jj];
+#endif
       }
       dsum = dsum + rowsum;
       for (int jj = 0; jj < 64; ++jj) p8[jj] = e4m3_encode(p[jj]);
       /* PV: two ordered K32 FP16 instantaneous buffers, each added in FP32 */
-      for (int sl = 0; sl < 2; ++sl) {
+#if ORACLE_PLANT == 12
+      const int SL = 64; /* planted: one K64 FP16 buffer instead of two K32 ones */
+#else
+      const int SL = 32;
+#endif
+      for (int sl = 0; sl < 64 / SL; ++sl) {
         for (int e = 0; e < D; ++e) {
           double acc = 0.0;
-          for (int jj = 32 * sl; jj < 32 * sl + 32; ++jj) {
+          for (int jj = SL * sl; jj < SL * sl + SL; ++jj) {
             int j = j0 + jj;
             if (j >= j1) break;
             acc += vdec[p8[jj]] * vdec[V[(int64_t)j * D + e]];
           }
+#if ORACLE_PLANT == 11
+          RO[e] = RO[e] + (float)acc; /* planted: FP16 buffer rounding skipped */
+#else
           RO[e] = RO[e] + f16_to_f32(f64_to_f16(acc));
+#endif
         }
       }
       m = m_new;

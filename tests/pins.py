@@ -6,8 +6,9 @@ deliberately wrong build of it, ``plant > 0``) disagrees with:
 * library conversions (E4M3 via ml_dtypes/torch, FP16 via NumPy, BF16 via
   torch) for the number formats;
 * the hand-worked four-token example in ``tests/golden``;
-* hand-worked group-boundary scales;
-* closed forms (Q = 0 gives the exact mean of exactly-representable V);
+* hand-worked group-boundary scales and half-way INT8 cases;
+* closed forms (Q = 0 gives the exact mean of exactly-representable V, and
+  the per-K32 FP16 buffers' roundings on hand-worked slice sums);
 * textbook FP64 softmax attention on small shapes (cosine and norm error);
 * invariants: K-offset invariance of the smoothed path, the online-softmax
   denominator, and dominance of one key;
@@ -362,7 +363,50 @@ def pin_norm_rope_exact(plant=0):
     assert np.array_equal(z2, 2.0 * y)
 
 
+def pin_int8_ties(plant=0):
+    """Half-way cases of the INT8 rule (hand-worked in the golden file): the
+    bytes of Q and K round to the even integer."""
+    with open(os.path.join(GOLDEN, "worked_int8_ties.json")) as f:
+        g = json.load(f)
+    N, H, D = 64, 1, 64
+    qf = np.zeros((N, H, D), np.float32)
+    kf = np.zeros((N, H, D), np.float32)
+    qc, kc = g["q_col0_rows0_9"], g["k_col0_rows0_11"]
+    qf[: len(qc), 0, 0] = qc
+    kf[: len(kc), 0, 0] = kc
+    q, k, v = make_qkv(qf, kf, np.zeros((N, H, D), np.float32))
+    qz = oracle.quantize(q, k, v, plant)
+    assert qz.q_scale[0, 0, 0] == 1.0 and qz.k_scale[0, 0, 0] == 1.0 and qz.k_mean[0, 0, 0] == 0.0
+    assert list(qz.q8[0, 0, : len(qc), 0]) == g["q_bytes_rows0_9"], qz.q8[0, 0, : len(qc), 0]
+    assert list(qz.k8[0, 0, : len(kc), 0]) == g["k_bytes_rows0_11"], qz.k8[0, 0, : len(kc), 0]
+
+
+def pin_f16_slice_buffers(plant=0):
+    """Closed form of the per-K32 FP16 buffers (hand-worked in the golden
+    file): with every probability exactly 1, RO is the in-order FP32 sum of
+    the FP16-rounded slice sums, chosen so that skipping the FP16 rounding or
+    merging the two slices of a tile changes the BF16 output."""
+    import torch
+    with open(os.path.join(GOLDEN, "worked_fp16_slices.json")) as f:
+        g = json.load(f)
+    N, H, D = g["n"], 1, 64
+    vf = np.zeros((N, H, D), np.float32)
+    for ch, col in g["v"].items():
+        for tok, val in col.items():
+            vf[int(tok), 0, int(ch)] = val
+    zero = np.zeros((N, H, D), np.float32)
+    q, k, v = make_qkv(zero, zero, vf)
+    qz = oracle.quantize(q, k, v, plant)
+    out = oracle.bf16_bits_to_float(oracle.attention(qz, 0.0, plant))[0, :, 0, :]
+    # the epilogue on the hand-worked RO: bf16(fl32(fl32(RO * fl32(1/d)) * 1))
+    rcp = np.float32(1.0) / np.float32(N)
+    want = np.zeros(D, np.float32)
+    for ch, ro in g["ro"].items():
+        want[int(ch)] = torch.tensor(np.float32(ro) * rcp).to(torch.bfloat16).float().item()
+    assert np.array_equal(out, np.broadcast_to(want, out.shape)), (out[0, :4], want[:4])
+
+
 ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_f16_round, pin_bf16_round, pin_worked_example,
             pin_group_boundaries, pin_q_zero_mean, pin_fp64_bruteforce, pin_dominance,
             pin_k_offset_invariance, pin_denominator, pin_qk_s32, pin_norm_rope_fp64,
-            pin_norm_rope_exact]
+            pin_norm_rope_exact, pin_int8_ties, pin_f16_slice_buffers]

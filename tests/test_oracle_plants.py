@@ -15,6 +15,13 @@ PLANTS = {
     7: "max not subtracted before exp2",
     8: "V scale not applied in the epilogue",
     9: "RoPE rotation sign flipped in the first half",
+    10: "denominator summed from the E4M3 probabilities",
+    11: "FP16 rounding of the K32 buffers skipped",
+    12: "one K64 FP16 buffer per tile instead of two K32 ones",
+    13: "keys past N in the last tile not masked",
+    14: "INT8 ties rounded away from zero",
+    15: "K mean taken over the 64-padded length",
+    16: "Q scale read per 64 rows in the score scale",
 }
 
 

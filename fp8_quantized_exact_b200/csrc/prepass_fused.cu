@@ -394,6 +394,18 @@ int sm_count() {
   return n;
 }
 
+// Work items of one call: the kernel's ticket counter and its item count are
+// int, and each CTA draws one ticket past the end before it leaves.
+constexpr long long kMaxItems = 1LL << 30;
+
+template <int D>
+long long fused_items(int B, int N, int H) {
+  constexpr int CPI = 128 / (D / 8);
+  const long long T64 = ceil_div(N, kKTile), Gq = ceil_div(N, kQTile) * kQTile / kQGroup;
+  const long long per_head = 2 * ((T64 + CPI - 1) / CPI) + (Gq + kQPerItem - 1) / kQPerItem;
+  return ((long long)B * H + kLookahead) * per_head;
+}
+
 template <int D>
 int fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N, int H,
           const FusedOut& o, cudaStream_t s) {
@@ -423,13 +435,19 @@ int fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16
   a.status = o.status;
   a.wait_limit = o.wait_limit;
   if (cudaMemsetAsync(o.counters, 0, sizeof(int) * (1 + 2 * (size_t)B * H), s) != cudaSuccess) return SAGE_ERR_CUDA;
-  const long long items = (long long)(B * H + kLookahead) * a.per_head;
+  const long long items = fused_items<D>(B, N, H);
+  if (items > kMaxItems) return SAGE_ERR_UNSUPPORTED;
   const int grid = (int)std::min<long long>(items, 2LL * sm_count());
   prepass_fused_kernel<D><<<grid, kThreadsP, 0, s>>>(a);
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 }  // namespace
+
+bool prepass_fused_fits(int B, int N, int H, int D) {
+  if (D != 64 && D != 128) return false;
+  return (D == 128 ? fused_items<128>(B, N, H) : fused_items<64>(B, N, H)) <= kMaxItems;
+}
 
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s) {

@@ -14,6 +14,7 @@ using namespace sage;
 namespace {
 
 constexpr size_t kAlign = 1024;
+constexpr int kMaxGridYZ = 65535;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 int g_mainloop = SAGE_MAINLOOP_DEFAULT;
@@ -37,6 +38,8 @@ Dims make_dims(int B, int N, int H, int D) {
 int check_dims(int B, int N, int H, int D) {
   if (B < 0 || N < 0 || H < 0 || D < 0) return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  // H and B are the y and z extents of the kernels' grids
+  if (B > kMaxGridYZ || H > kMaxGridYZ) return SAGE_ERR_UNSUPPORTED;
   // keep every flat index inside int range assumptions of the kernels
   if ((int64_t)B * H > (1 << 30) || N > (1 << 28)) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
@@ -348,6 +351,7 @@ int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, 
   int rc = check_dims(B, N, H, D);
   if (rc) return rc;
   if (empty(B, N, H)) return SAGE_OK;
+  if (!prepass_fused_fits(B, N, H, D)) return SAGE_ERR_UNSUPPORTED;
   if ((rc = check_view(q)) || (rc = check_view(k)) || (rc = check_view(v))) return rc;
   if (!q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean || !v_fp8 || !v_scale) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(q_scale) || !aligned16(k_scale) ||

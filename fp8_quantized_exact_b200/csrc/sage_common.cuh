@@ -129,6 +129,9 @@ int launch_norm_rope_qk(const NormRopeIn& in, const sage_view_bf16& q, const sag
                         int D, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean, double* k_part,
                         cudaStream_t s);
 void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s);
+// false when the single-launch prepass would need more work items than its
+// int ticket counter allows (B*H*N beyond about 1.8e11)
+bool prepass_fused_fits(int B, int N, int H, int D);
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s);
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,

@@ -33,6 +33,9 @@
  *     streams the caller passes to sage_attn_fwd_host.
  *   - Shapes: B (batch), N (tokens), H (heads), D (head dim, 64 or 128).
  *     B, N or H equal to 0 is an empty problem: SAGE_OK, nothing launched.
+ *     Limits (SAGE_ERR_UNSUPPORTED beyond them): B <= 65535 and H <= 65535
+ *     (grid extents), B*H <= 2^30, N <= 2^28; sage_quant_qkv also needs
+ *     B*H*N below about 1.8e11 (D = 128) or 2.7e11 (D = 64).
  *   - BF16 views carry element strides (b, n, h); d has unit stride.  The
  *     base address and every stride must be 16-byte aligned (strides a
  *     multiple of 8 elements); three views may alias one fused projection
@@ -73,7 +76,8 @@ extern "C" {
 enum sage_status_code {
   SAGE_OK = 0,
   SAGE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad stride */
-  SAGE_ERR_UNSUPPORTED = 2,  /* D not in {64, 128}; misaligned base or stride */
+  SAGE_ERR_UNSUPPORTED = 2,  /* D not in {64, 128}; misaligned base or stride;
+                                a size beyond the limits below */
   SAGE_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or too small */
   SAGE_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
   SAGE_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out */

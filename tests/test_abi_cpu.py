@@ -61,6 +61,10 @@ def test_argument_errors_need_no_device(lib):
     assert lib.sage_workspace_bytes(2, 1, 100, 2, 96, ctypes.byref(n)) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_workspace_bytes(2, -1, 100, 2, 64, ctypes.byref(n)) == sage.SAGE_ERR_INVALID_ARG
     assert lib.sage_workspace_bytes(9, 1, 100, 2, 64, ctypes.byref(n)) == sage.SAGE_ERR_INVALID_ARG
+    # grid extents: B and H at most 65535 each; B*H at most 2^30; N at most 2^28
+    for (B, N, H) in ((65536, 16, 1), (1, 16, 65536), (32768, 16, 32769), (1, (1 << 28) + 1, 1)):
+        assert lib.sage_workspace_bytes(2, B, N, H, 64, ctypes.byref(n)) == sage.SAGE_ERR_UNSUPPORTED, (B, N, H)
+    assert lib.sage_workspace_bytes(2, 65535, 16, 1, 64, ctypes.byref(n)) == sage.SAGE_OK
     null = sage.sage_view_bf16(None, 0, 0, 0)
     good = sage.sage_view_bf16(4096, 256 * 2 * 128, 2 * 128, 128)
     odd = sage.sage_view_bf16(4096 + 2, 256 * 2 * 128, 2 * 128, 128)
@@ -97,6 +101,11 @@ def test_argument_errors_need_no_device(lib):
                None) == sage.SAGE_ERR_INVALID_ARG
     assert qkv(v4, v4, v4, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 100,
                None) == sage.SAGE_ERR_WORKSPACE
+    # the single-launch prepass's int work-item counter: 2^14 heads of 2^24 tokens need too many items
+    assert qkv(v4, v4, v4, 1, 1 << 24, 1 << 14, 128, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+               None) == sage.SAGE_ERR_UNSUPPORTED
+    assert qkv(v4, v4, v4, 70000, 10, 1, 64, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
+               None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_set_mainloop(7) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_set_mainloop(-1) == sage.SAGE_ERR_UNSUPPORTED
     # every declared mainloop value is accepted; the explicit ones read back as set

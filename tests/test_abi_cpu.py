@@ -140,3 +140,51 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sage, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         sage.lib()
+
+
+def test_header_compiles_as_c_and_links(lib, tmp_path):
+    """The header is plain C: a C99 program that includes it, takes the
+    address of every declared function and calls the argument-only entry
+    points compiles with -pedantic -Werror, links against the library and
+    runs without a GPU."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = sorted(declared_functions())
+    table = ",\n    ".join(f"(void (*)(void))&{n}" for n in names)
+    src = tmp_path / "abi_check.c"
+    src.write_text(f"""#include <stdio.h>
+#include <string.h>
+#include "sage_b200.h"
+
+static void (*const every_entry[])(void) = {{
+    {table}
+}};
+
+int main(void) {{
+  size_t bytes = 0;
+  sage_fwd_layout lay;
+  unsigned i;
+  for (i = 0; i < sizeof every_entry / sizeof every_entry[0]; ++i)
+    if (!every_entry[i]) return 10;
+  if (sage_workspace_bytes(SAGE_OP_ATTN_FWD, 1, 1000, 8, 128, &bytes) != SAGE_OK || bytes == 0) return 1;
+  if (sage_fwd_workspace_layout(1, 1000, 8, 128, &lay) != SAGE_OK || lay.total != bytes) return 2;
+  if (sage_workspace_bytes(SAGE_OP_ATTN_FWD, 1, 1000, 8, 96, &bytes) != SAGE_ERR_UNSUPPORTED) return 3;
+  if (sage_workspace_bytes(SAGE_OP_ATTN_FWD, 1, 1000, 8, 128, NULL) != SAGE_ERR_INVALID_ARG) return 4;
+  if (strcmp(sage_strerror(SAGE_OK), "success") != 0) return 5;
+  if (sage_set_mainloop(99) != SAGE_ERR_UNSUPPORTED) return 6;
+  printf("%u entry points\\n", i);
+  return 0;
+}}
+""")
+    so = os.path.abspath(lib._name)
+    exe = tmp_path / "abi_check"
+    cc = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror", "-I",
+                         os.path.join(ROOT, "include"), str(src), so, f"-Wl,-rpath,{os.path.dirname(so)}",
+                         "-o", str(exe)], capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert run.stdout.strip() == f"{len(names)} entry points"

@@ -384,13 +384,13 @@ __global__ void __launch_bounds__(kThreadsP, 2) prepass_fused_kernel(const Fused
   }
 }
 
+// SM count of the current device (asked on every call: the runtime answers
+// from its own cache, and devices of one process may differ)
 int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      n = 148;
-  }
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    n = 148;
   return n;
 }
 

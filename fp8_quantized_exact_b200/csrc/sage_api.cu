@@ -5,6 +5,8 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 #include <vector>
 
 #include "sage_common.cuh"
@@ -17,10 +19,11 @@ constexpr size_t kAlign = 1024;
 constexpr int kMaxGridYZ = 65535;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-int g_mainloop = SAGE_MAINLOOP_DEFAULT;
-bool g_mainloop_env_read = false;
-int g_stall_tile = -1;                        // test hook (sage_debug_set_stall)
-long long g_wait_limit = kDefaultWaitLimit;
+// Process-wide settings; entry points may be called from several threads.
+std::atomic<int> g_mainloop{SAGE_MAINLOOP_DEFAULT};
+std::once_flag g_mainloop_env_once;            // SAGE_MAINLOOP is read once
+std::atomic<int> g_stall_tile{-1};             // test hook (sage_debug_set_stall)
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 struct Dims {
   int B, N, H, D, Nq, Nk, G32, T64;
@@ -121,7 +124,7 @@ FusedOut fused_out(void* ws, const Layout& L, int8_t* q8, float* qs, int8_t* k8,
   o.v_part = at<float>(ws, L.v_part);
   o.counters = at<int>(ws, L.counters);
   o.status = static_cast<DeviceStatus*>(ws);
-  o.wait_limit = g_wait_limit;
+  o.wait_limit = g_wait_limit.load();
   return o;
 }
 
@@ -134,18 +137,21 @@ float log2_scale(float sm_scale, int D) {
   return (float)((double)sm_scale * 1.4426950408889634074);
 }
 
+// The SAGE_MAINLOOP environment variable picks the mainloop until the first
+// sage_set_mainloop call, which always wins.
+void read_mainloop_env() {
+  const char* e = getenv("SAGE_MAINLOOP");
+  if (!e) return;
+  if (!strcmp(e, "tcgen05")) g_mainloop.store(SAGE_MAINLOOP_TCGEN05);
+  else if (!strcmp(e, "mma_sync") || !strcmp(e, "mmasync")) g_mainloop.store(SAGE_MAINLOOP_MMA_SYNC);
+  else if (!strcmp(e, "tcgen05_f32")) g_mainloop.store(SAGE_MAINLOOP_TCGEN05_F32);
+}
+
 int resolved_mainloop() {
-  if (!g_mainloop_env_read) {
-    g_mainloop_env_read = true;
-    const char* e = getenv("SAGE_MAINLOOP");
-    if (e && g_mainloop == SAGE_MAINLOOP_DEFAULT) {
-      if (!strcmp(e, "tcgen05")) g_mainloop = SAGE_MAINLOOP_TCGEN05;
-      else if (!strcmp(e, "mma_sync") || !strcmp(e, "mmasync")) g_mainloop = SAGE_MAINLOOP_MMA_SYNC;
-      else if (!strcmp(e, "tcgen05_f32")) g_mainloop = SAGE_MAINLOOP_TCGEN05_F32;
-    }
-  }
-  if (g_mainloop == SAGE_MAINLOOP_DEFAULT) return tc_available() ? SAGE_MAINLOOP_TCGEN05 : SAGE_MAINLOOP_MMA_SYNC;
-  return g_mainloop;
+  std::call_once(g_mainloop_env_once, read_mainloop_env);
+  const int m = g_mainloop.load();
+  if (m == SAGE_MAINLOOP_DEFAULT) return tc_available() ? SAGE_MAINLOOP_TCGEN05 : SAGE_MAINLOOP_MMA_SYNC;
+  return m;
 }
 
 AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const int8_t* k8,
@@ -159,8 +165,8 @@ AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const i
   p.Nq = d.Nq; p.Nk = d.Nk; p.G32 = d.G32; p.T64 = d.T64;
   p.sl2 = log2_scale(sm_scale, d.D);
   p.status = static_cast<DeviceStatus*>(status);
-  p.wait_limit = g_wait_limit;
-  p.stall_tile = g_stall_tile;
+  p.wait_limit = g_wait_limit.load();
+  p.stall_tile = g_stall_tile.load();
   return p;
 }
 
@@ -512,16 +518,16 @@ const char* sage_strerror(int code) {
 
 int sage_set_mainloop(int which) {
   if (which < SAGE_MAINLOOP_DEFAULT || which > SAGE_MAINLOOP_TCGEN05_F32) return SAGE_ERR_UNSUPPORTED;
-  g_mainloop = which;
-  g_mainloop_env_read = true;
+  std::call_once(g_mainloop_env_once, read_mainloop_env);
+  g_mainloop.store(which);
   return SAGE_OK;
 }
 
 int sage_get_mainloop(void) { return resolved_mainloop(); }
 
 int sage_debug_set_stall(int k_tile, long long wait_limit_cycles) {
-  g_stall_tile = k_tile < 0 ? -1 : k_tile;
-  g_wait_limit = wait_limit_cycles > 0 ? wait_limit_cycles : kDefaultWaitLimit;
+  g_stall_tile.store(k_tile < 0 ? -1 : k_tile);
+  g_wait_limit.store(wait_limit_cycles > 0 ? wait_limit_cycles : kDefaultWaitLimit);
   return SAGE_OK;
 }
 

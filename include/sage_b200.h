@@ -267,7 +267,10 @@ SAGE_API int sage_read_device_status(const void* workspace, void* stream);
 SAGE_API const char* sage_strerror(int code);
 
 /* Select the mainloop used by sage_attn_fwd / sage_attn_from_quant for the
- * calling process.  Returns SAGE_ERR_UNSUPPORTED for an unknown value. */
+ * calling process.  Returns SAGE_ERR_UNSUPPORTED for an unknown value.
+ * Until the first call, the environment variable SAGE_MAINLOOP ("tcgen05",
+ * "mma_sync" or "tcgen05_f32", read once) may pick it.  Safe to call from
+ * several threads; a launch uses the value current when it is enqueued. */
 SAGE_API int sage_set_mainloop(int which);
 SAGE_API int sage_get_mainloop(void);
 

@@ -1,4 +1,4 @@
-"""Ulysses head-sharded attention with two gloo ranks on CPU: the exchange
+"""Ulysses head-sharded attention with two and four gloo ranks on CPU: the exchange
 layout (token shards -> head shards -> token shards, ragged token counts,
 strided inputs) gives every rank exactly the rows the single-process
 computation gives for its tokens.  The local attention here is the oracle's
@@ -27,6 +27,8 @@ def _inputs(case):
     import synth
     if case == "ragged":
         return synth.custom(1, 300, 4, 64, seed=17), [137, 163]
+    if case == "four_ranks":  # batch of 2, one rank without tokens, 2 heads per rank
+        return synth.custom(2, 160, 8, 64, seed=19), [50, 0, 77, 33]
     return synth.make_inputs(synth.Config("fused_small", 1, 200, 2, 128, layout="fused_qkv"), seed=18), [100, 100]
 
 
@@ -59,19 +61,20 @@ def _worker(rank, world, port, case, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("case", ["ragged", "fused"])
-def test_two_rank_ulysses_matches_single_process(case):
+@pytest.mark.parametrize("case", ["ragged", "fused", "four_ranks"])
+def test_ulysses_matches_single_process(case):
     import oracle
-    ctx = mp.get_context("spawn")
-    with ctx.Manager() as mgr:
-        out = mgr.dict()
-        mp.start_processes(_worker, args=(2, _free_port(), case, out), nprocs=2, join=True, start_method="spawn")
-        res = dict(out)
     inp, counts = _inputs(case)
+    world = len(counts)
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_worker, args=(world, _free_port(), case, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
     ref = oracle.attention(oracle.quantize(inp.q, inp.k, inp.v))
     o = 0
-    for r in range(2):
+    for r in range(world):
         got = res[r]
-        assert got.shape == (1, counts[r]) + inp.q.shape[2:]
+        assert got.shape == (inp.q.shape[0], counts[r]) + inp.q.shape[2:]
         assert np.array_equal(got, ref[:, o:o + counts[r]]), f"rank {r} differs"
         o += counts[r]

@@ -188,3 +188,37 @@ int main(void) {{
     run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert run.stdout.strip() == f"{len(names)} entry points"
+
+
+def _header_prototypes():
+    protos = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if not fn.endswith(".h"):
+            continue
+        with open(os.path.join(ROOT, "include", fn)) as f:
+            text = re.sub(r"/\*.*?\*/", " ", f.read(), flags=re.S)
+        for ret, name, params in re.findall(r"SAGE_API\s+([\w\s\*]+?)\s*\b(sage_\w+)\s*\(([^)]*)\)\s*;", text):
+            plist = [p.strip() for p in params.split(",")]
+            if plist == ["void"]:
+                plist = []
+            protos[name] = (" ".join(ret.split()), [re.sub(r"\s*\b\w+$", "", p).strip() for p in plist])
+    return protos
+
+
+def test_binding_signatures_match_the_header(lib):
+    """Every ctypes prototype the binding sets has the header's parameter
+    count and kinds, and the header's return type."""
+    scalar = {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "size_t": ctypes.c_size_t,
+              "long long": ctypes.c_longlong, "float": ctypes.c_float, "sage_view_bf16": sage.sage_view_bf16}
+    protos = _header_prototypes()
+    assert set(protos) == set(sage.EXPORTS)
+    for name, (ret, params) in protos.items():
+        f = getattr(lib, name)
+        assert len(f.argtypes) == len(params), (name, len(f.argtypes), params)
+        for i, (ctype, decl) in enumerate(zip(f.argtypes, params)):
+            if "*" in decl:
+                assert ctype is ctypes.c_void_p or issubclass(ctype, ctypes._Pointer), (name, i, decl, ctype)
+            else:
+                assert ctype is scalar[decl], (name, i, decl, ctype)
+        want = ctypes.c_char_p if ret == "const char*" else scalar[ret]
+        assert f.restype is want, (name, ret, f.restype)

@@ -222,3 +222,22 @@ def test_binding_signatures_match_the_header(lib):
                 assert ctype is scalar[decl], (name, i, decl, ctype)
         want = ctypes.c_char_p if ret == "const char*" else scalar[ret]
         assert f.restype is want, (name, ret, f.restype)
+
+
+def test_product_path_does_not_reach_the_oracle(lib):
+    """The library and its binding neither import, load nor link anything of
+    the oracle; the oracle's C source includes nothing of the library."""
+    import subprocess
+    pkg = os.path.join(ROOT, "fp8_quantized_exact_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".c")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    text = f.read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b|liboracle|sage_oracle|oracle_\w+\(", text, re.M), fn
+    needed = subprocess.run(["readelf", "-d", sage.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in needed and "synth" not in needed
+    with open(os.path.join(ROOT, "oracle", "sage_oracle.c")) as f:
+        src = f.read()
+    assert not re.search(r'#include\s+"', src), "the oracle includes a project header"
+    assert "sage_b200" not in src and "csrc" not in src

@@ -1,7 +1,8 @@
 """Host logic of bench.py that needs no GPU: the reference arm sizes each
 timed step's oracle sample from the costs its first warm-up step measures,
 so that all timed steps fit the budget, and prints one JSON line with the
-contract's keys."""
+contract's keys; the clock record of a timed region is summarised and a
+slowdown voids its number."""
 import argparse
 import json
 import os
@@ -61,3 +62,27 @@ def test_reference_arm_prints_nothing_on_other_ranks(monkeypatch, capsys):
     monkeypatch.setattr(bench, "cpu_sample", lambda *a: pytest.fail("rank 1 must not sample"))
     bench.run_reference(_args(3), synth.CONFIGS["small"], 1, 2)
     assert capsys.readouterr().out == ""
+
+
+def _smi(mhz, reasons=()):
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    flags = ["Active" if n in reasons else "Not Active" for n in names]
+    return f"0, {mhz}, 1965, 900.00, 0x0000000000000000, " + ", ".join(flags) + "\n"
+
+
+def test_clock_summary_and_rejection():
+    # an idle sample before the load is left out of the median; reasons seen anywhere count
+    s = bench.summarize_clocks([_smi(345), _smi(1965), _smi(1950), _smi(1965)])
+    assert s == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 4, "reasons": []}
+    assert bench.clocks_rejection(s) is None
+    # a power cap alone is kept, even at lower clocks
+    s = bench.summarize_clocks([_smi(1310, ["sw_power_cap"])] * 3)
+    assert s["reasons"] == ["sw_power_cap"] and bench.clocks_rejection(s) is None
+    # any hardware or thermal slowdown voids the number
+    s = bench.summarize_clocks([_smi(1965), _smi(1800, ["hw_thermal_slowdown"])])
+    assert bench.clocks_rejection(s) == "hw_thermal_slowdown"
+    # clocks held low with no reason: a leftover clock lock
+    s = bench.summarize_clocks([_smi(1200)] * 5)
+    assert bench.clocks_rejection(s) == "sm clock held low with no reason"
+    # no samples (sampling off or nvidia-smi missing): nothing to judge
+    assert bench.summarize_clocks(["garbage\n"]) is None and bench.clocks_rejection(None) is None

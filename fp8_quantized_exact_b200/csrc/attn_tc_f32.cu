@@ -24,8 +24,8 @@
 //   warps 8-11  correction and epilogue owners, one per quadrant: per tile
 //               they wait for its probabilities and for the previous tile's
 //               PV MMAs (one barrier per tile mod 4); on a tile whose flag is
-//               set they scale the FP32 accumulator rows by r in TMEM; then
-//               they release the tile's PV; at the end they apply 1/d and the
+//               set they scale the FP32 accumulator rows by r in TMEM and then
+//               release that tile's PV MMAs; at the end they apply 1/d and the
 //               V scale and store BF16.
 //   warp 12     TMA producer (K and V^T stages of 128 keys).
 //   warp 13     QK issuer (N = 128 per 128-key group, two score buffers).

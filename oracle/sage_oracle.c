@@ -428,8 +428,10 @@ int oracle_attn_rows(const int8_t* q8, const float* q_scale, const int8_t* k8, c
       /* update_mdo: new max, ro_rescale applied to RO and d */
       const float m_new = m > tmax ? m : tmax;
       const float r = (float)exp2((double)(m - m_new));
-#if ORACLE_PLANT != 6
+#if ORACLE_PLANT != 6 && ORACLE_PLANT != 17 && ORACLE_PLANT != 18
       for (int e = 0; e < D; ++e) RO[e] = RO[e] * r;
+#endif
+#if ORACLE_PLANT != 6
       dsum = dsum * r;
 #endif
       /* accumulate_d on FP32 probabilities, then RS_32_to_8 */
@@ -470,6 +472,9 @@ int oracle_attn_rows(const int8_t* q8, const float* q_scale, const int8_t* k8, c
 #endif
         }
       }
+#if ORACLE_PLANT == 17
+      for (int e = 0; e < D; ++e) RO[e] = RO[e] * r; /* planted: RO rescaled after the tile's PV */
+#endif
       m = m_new;
     }
     /* final normalisation: FP32 reciprocal of d, then the V scale, then BF16 */

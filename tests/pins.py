@@ -12,6 +12,8 @@ deliberately wrong build of it, ``plant > 0``) disagrees with:
 * textbook FP64 softmax attention on small shapes (cosine and norm error);
 * invariants: K-offset invariance of the smoothed path, the online-softmax
   denominator, and dominance of one key;
+* the online softmax against the global-maximum form, bit for bit, where
+  every rescale is an exact power of two;
 * brute-force integer QK^T via NumPy.
 
 They are collected by ``test_oracle_pins.py``; ``test_oracle_plants.py``
@@ -406,7 +408,84 @@ def pin_f16_slice_buffers(plant=0):
     assert np.array_equal(out, np.broadcast_to(want, out.shape)), (out[0, :4], want[:4])
 
 
+# ------------------------------------------------ online softmax, exactly
+def _rising_max_inputs(N, seed):
+    """Q, K, V for which every score is an integer in log2 units and each
+    64-key tile raises every row's running maximum by exactly one.
+
+    The score scale is exactly 1: sm_scale = fl32(ln 2) gives
+    fl32(sm_scale * log2 e) = 1, and every Q group and K block has amax 127
+    (one entry of 127 in a column that meets only zeros on the other side),
+    so q_scale = k_scale = 1 and the bytes are the values themselves.  K
+    column 0 carries the scores: tile t holds one key of value t and others
+    in [t - 4, t - 2]; its mean is made an integer, so smoothing keeps every
+    byte integral.  Q column 1 and K column 1 (zero mean, +-1) make the rows
+    differ.  Every score lies within 8 of the row's final maximum, so every
+    probability is a power of two that E4M3 holds exactly.  V is drawn from
+    {0, +-1, +-2, +-4} with amax 4, whose E4M3 codes are exact."""
+    rng = np.random.default_rng(seed)
+    D, T = 64, -(-N // 64)
+    qf = np.zeros((N, 1, D), np.float32)
+    kf = np.zeros((N, 1, D), np.float32)
+    qf[:, 0, 0] = 1.0
+    qf[:, 0, 1] = rng.integers(0, 2, N)
+    qf[::32, 0, 2] = 127.0
+    tile = np.arange(N) // 64
+    star = np.arange(N) % 64 == 0
+    t = rng.integers(tile - 4, tile - 1)
+    t[star] = tile[star]
+    excess = t.sum() % N                       # lower non-maximum keys until the mean is integral
+    for j in np.flatnonzero(~star & (t > tile - 4))[:excess]:
+        t[j] -= 1
+    assert t.sum() % N == 0, "not enough keys to adjust"
+    kf[:, 0, 0] = t
+    k1 = rng.integers(-1, 2, N)
+    k1[star] = 0
+    for j in np.flatnonzero(~star):            # zero mean: move keys towards 0 until balanced
+        if k1.sum() == 0:
+            break
+        if k1[j] != 0 and np.sign(k1[j]) == np.sign(k1.sum()):
+            k1[j] = 0
+    assert k1.sum() == 0
+    kf[:, 0, 1] = k1
+    kf[star, 0, 3] = 127.0
+    kf[np.flatnonzero(star) + 1, 0, 3] = -127.0
+    vf = rng.choice(np.array([0, 1, -1, 2, -2, 4, -4], np.float32), size=(N, 1, D))
+    vf[0] = 4.0
+    return qf, kf, vf
+
+
+def pin_online_rescale_exact(plant=0):
+    """With power-of-two rescales the online softmax must equal, bit for bit,
+    the same arithmetic done once against the global row maximum: every
+    rescale r = 2^-1 is exact, as is its effect on the E4M3 probabilities,
+    the FP16 slice sums, the FP32 accumulator and the denominator.  The
+    global form here is NumPy and torch conversions only."""
+    import torch
+    sm = np.float32(np.log(2.0))
+    for N in (256, 230, 100):
+        qf, kf, vf = _rising_max_inputs(N, 7 + N)
+        q, k, v = make_qkv(qf, kf, vf)
+        qz = oracle.quantize(q, k, v, plant)
+        got = oracle.attention(qz, float(sm), plant)[0, :, 0, :]
+        S = qz.q8[0, 0].astype(np.int64) @ qz.k8[0, 0].astype(np.int64).T
+        tmax = [S[:, j:j + 64].max(axis=1) for j in range(0, N, 64)]
+        assert all(np.all(b == a + 1) for a, b in zip(tmax, tmax[1:])), "inputs: maxima must rise by one"
+        e = S - S.max(axis=1, keepdims=True)
+        assert e.min() >= -9, "inputs: a probability would underflow E4M3"
+        p = np.ldexp(1.0, e)
+        p8 = torch.from_numpy(p.astype(np.float32)).to(torch.float8_e4m3fn).double().numpy()
+        v8 = torch.from_numpy(np.ascontiguousarray(qz.v8[0, 0])).view(torch.float8_e4m3fn).double().numpy()
+        RO = np.zeros(got.shape, np.float32)
+        for j0 in range(0, N, 32):  # K32 slices in order: FP16 sum, then the FP32 add
+            RO = RO + (p8[:, j0:j0 + 32] @ v8[j0:j0 + 32]).astype(np.float16).astype(np.float32)
+        rcp = np.float32(1.0) / p.sum(axis=1).astype(np.float32)
+        o = (RO * rcp[:, None]) * qz.v_scale[0, 0][None, :]
+        want = torch.from_numpy(o.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got, want), (N, int((got != want).sum()))
+
+
 ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_f16_round, pin_bf16_round, pin_worked_example,
             pin_group_boundaries, pin_q_zero_mean, pin_fp64_bruteforce, pin_dominance,
             pin_k_offset_invariance, pin_denominator, pin_qk_s32, pin_norm_rope_fp64,
-            pin_norm_rope_exact, pin_int8_ties, pin_f16_slice_buffers]
+            pin_norm_rope_exact, pin_int8_ties, pin_f16_slice_buffers, pin_online_rescale_exact]

@@ -22,6 +22,8 @@ PLANTS = {
     14: "INT8 ties rounded away from zero",
     15: "K mean taken over the 64-padded length",
     16: "Q scale read per 64 rows in the score scale",
+    17: "accumulator rescaled after the tile's PV instead of before",
+    18: "accumulator not rescaled (the denominator is)",
 }
 
 

@@ -241,3 +241,19 @@ def test_product_path_does_not_reach_the_oracle(lib):
         src = f.read()
     assert not re.search(r'#include\s+"', src), "the oracle includes a project header"
     assert "sage_b200" not in src and "csrc" not in src
+
+
+def test_long_context_tile_geometry(lib):
+    """The pages' tiling of the 37,810-token workload: 591 key tiles of 64,
+    296 query tiles of 128 (the (296, 56, 1) grid) and so 1,182 query groups
+    of 32 ("Vortex Exact Attention", section "Authoritative Baseline";
+    "architecture_model.json", key "baseline"; "State-Ownership Architecture
+    Decision", section "Non-Negotiable Dataflow"); the workspace holds
+    those padded buffers."""
+    shp = sage.quant_shapes(1, 37810, 56, 128)
+    assert shp["k_scale"] == (1, 56, 591) and shp["q_scale"] == (1, 56, 1182)
+    assert shp["q_i8"] == (1, 56, 296 * 128, 128) and shp["v_fp8"] == (1, 56, 128, 591 * 64)
+    lay = sage.sage_fwd_workspace_layout(1, 37810, 56, 128)
+    assert lay["q_scale"] - lay["q_i8"] >= 56 * 296 * 128 * 128
+    assert lay["k_scale"] - lay["k_i8"] >= 56 * 591 * 64 * 128
+    assert lay["v_scale"] - lay["v_fp8"] >= 56 * 128 * 591 * 64

@@ -237,13 +237,16 @@ def _sampled_rows(N):
 def test_full_size_sampled_parity(sage, dev, cfg):
     """Full-size workloads in the benchmark's launch configuration: bytes and
     scales of two sampled heads bit-exact, output rows of three 32-row query
-    groups per sampled head (first, middle, last/ragged) within tolerance."""
+    groups per sampled head (first, middle, last/ragged) within tolerance,
+    and every output element finite."""
     c = synth.CONFIGS[cfg]
     inp = synth.make_inputs(c, seed=0)
     (q, k, v), _ = gu.to_device(inp, dev)
     heads = [(0, 0), (c.B - 1, c.H - 1)]
     for ml in mainloops():
         out, ws = gu.run_fwd(sage, q, k, v, ml)
+        # a property of every row: no NaN or infinity anywhere in the output
+        assert bool(torch.isfinite(out).all()), f"{cfg} ml={ml}: non-finite output"
         got = gu.logical_quant(sage, ws, c.B, c.N, c.H, c.D, heads=heads)
         outh = out.float().cpu().numpy()
         for i, (b, h) in enumerate(heads):

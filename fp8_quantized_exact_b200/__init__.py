@@ -12,7 +12,6 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_build", "libsage_b200.so")

@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", default="long_fused")
+    ap.add_argument("--config", default="long_fused",
+                    choices=["small", "ragged", "outlier", "long_fused", "d64_batch"])
     ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=4)

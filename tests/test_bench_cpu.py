@@ -86,3 +86,19 @@ def test_clock_summary_and_rejection():
     assert bench.clocks_rejection(s) == "sm clock held low with no reason"
     # no samples (sampling off or nvidia-smi missing): nothing to judge
     assert bench.summarize_clocks(["garbage\n"]) is None and bench.clocks_rejection(None) is None
+
+
+def test_defaults_follow_the_contract(monkeypatch):
+    # no flags: one GPU, the long-context workload, at least 3 warm-up steps,
+    # every mainloop and workload name accepted
+    monkeypatch.setattr(sys, "argv", ["bench.py"])
+    a = bench.parse()
+    assert (a.gpus, a.config, a.impl, a.mainloop) == (1, "long_fused", "ours", "default")
+    assert a.warmup >= 3 and a.steps >= 1
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--config", "nonesuch"])
+    with pytest.raises(SystemExit):
+        bench.parse()
+    import synth
+    for name in synth.CONFIG_ORDER:
+        monkeypatch.setattr(sys, "argv", ["bench.py", "--config", name])
+        assert bench.parse().config == name

@@ -14,7 +14,11 @@ Every function takes and returns *logical* layouts:
 * ``v8``: uint8 E4M3 bytes ``[B, H, N, D]`` (token-major)
 * outputs: uint16 BF16 bits ``[rows, D]``
 
-Parity pins for each function live in ``tests/test_oracle_pins.py``.
+The pins that tie each function to facts outside it (library conversions,
+hand-worked examples, closed forms, FP64 attention, invariants, an exact
+global-maximum form) live in ``tests/pins.py``; ``tests/test_oracle_pins.py``
+runs them and ``tests/test_oracle_plants.py`` shows that each planted
+mistake (``ORACLE_PLANT``) fails one.
 """
 from __future__ import annotations
 

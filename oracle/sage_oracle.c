@@ -205,11 +205,21 @@ int oracle_k_mean(const uint16_t* k, int64_t sb, int64_t sn, int64_t sh,
   for (int b = 0; b < B; ++b)
     for (int h = 0; h < H; ++h)
       for (int d = 0; d < D; ++d) {
+#if ORACLE_PLANT == 19
+        float total = 0.0f; /* planted: the sums kept in FP32 */
+#else
         double total = 0.0;
+#endif
         for (int c0 = 0; c0 < N; c0 += 64) {
+#if ORACLE_PLANT == 19
+          float part = 0.0f;
+          int c1 = c0 + 64 < N ? c0 + 64 : N;
+          for (int n = c0; n < c1; ++n) part += bf16_to_f32(k[IDX_IN(b, n, h) + d]);
+#else
           double part = 0.0;
           int c1 = c0 + 64 < N ? c0 + 64 : N;
           for (int n = c0; n < c1; ++n) part += (double)bf16_to_f32(k[IDX_IN(b, n, h) + d]);
+#endif
           total += part;
         }
 #if ORACLE_PLANT == 1

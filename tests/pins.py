@@ -14,7 +14,8 @@ deliberately wrong build of it, ``plant > 0``) disagrees with:
   denominator, and dominance of one key;
 * the online softmax against the global-maximum form, bit for bit, where
   every rescale is an exact power of two;
-* brute-force integer QK^T via NumPy.
+* brute-force integer QK^T via NumPy;
+* the K channel mean against the correctly rounded mean of the exact sum.
 
 They are collected by ``test_oracle_pins.py``; ``test_oracle_plants.py``
 checks that each planted mistake fails at least one of them.
@@ -388,6 +389,16 @@ def pin_f16_slice_buffers(plant=0):
     file): with every probability exactly 1, RO is the in-order FP32 sum of
     the FP16-rounded slice sums, chosen so that skipping the FP16 rounding or
     merging the two slices of a tile changes the BF16 output."""
+    q, k, v, want = f16_slice_case()
+    qz = oracle.quantize(q, k, v, plant)
+    out = oracle.bf16_bits_to_float(oracle.attention(qz, 0.0, plant))[0, :, 0, :]
+    assert np.array_equal(out, np.broadcast_to(want, out.shape)), (out[0, :4], want[:4])
+
+
+def f16_slice_case():
+    """Inputs of the hand-worked FP16-slice fixture (B=1, N=104, H=1, D=64 BF16
+    bits) and its expected output row (every row is the same): the epilogue
+    bf16(fl32(fl32(RO * fl32(1/d)) * 1)) applied to the hand-worked RO."""
     import torch
     with open(os.path.join(GOLDEN, "worked_fp16_slices.json")) as f:
         g = json.load(f)
@@ -398,14 +409,11 @@ def pin_f16_slice_buffers(plant=0):
             vf[int(tok), 0, int(ch)] = val
     zero = np.zeros((N, H, D), np.float32)
     q, k, v = make_qkv(zero, zero, vf)
-    qz = oracle.quantize(q, k, v, plant)
-    out = oracle.bf16_bits_to_float(oracle.attention(qz, 0.0, plant))[0, :, 0, :]
-    # the epilogue on the hand-worked RO: bf16(fl32(fl32(RO * fl32(1/d)) * 1))
     rcp = np.float32(1.0) / np.float32(N)
     want = np.zeros(D, np.float32)
     for ch, ro in g["ro"].items():
         want[int(ch)] = torch.tensor(np.float32(ro) * rcp).to(torch.bfloat16).float().item()
-    assert np.array_equal(out, np.broadcast_to(want, out.shape)), (out[0, :4], want[:4])
+    return q, k, v, want
 
 
 # ------------------------------------------------ online softmax, exactly
@@ -485,7 +493,46 @@ def pin_online_rescale_exact(plant=0):
         assert np.array_equal(got, want), (N, int((got != want).sum()))
 
 
+# ------------------------------------------------------------ K mean (R1)
+def f32_nearest(fr):
+    """A Fraction rounded to the nearest float32, ties to even (exact: the
+    float64 value from the correctly rounded Fraction division only brackets
+    the answer; the Fraction comparison decides it)."""
+    from fractions import Fraction
+    x = np.float32(float(fr))
+    cands = {x, np.nextafter(x, np.float32(np.inf)), np.nextafter(x, np.float32(-np.inf))}
+    best = min(cands, key=lambda c: (abs(Fraction(float(c)) - fr), int(np.array(c).view(np.uint32)) & 1))
+    return np.float32(best)
+
+
+def pin_k_mean_exact(plant=0):
+    """Reading R1 without trusting its summation order: on random BF16 K of
+    37,810 tokens (the long-context length) with per-channel offsets of up to
+    2^10 and N(0,1) noise, every channel mean equals float32(sum / N) of the
+    exact rational sum, rounded once to nearest even.  The sum is exact in
+    FP64 for these values (they span fewer than 53 bits), so the FP64 reading
+    meets it; a sum kept in FP32 does not."""
+    from fractions import Fraction
+    N, D = 37810, 128
+    rng = np.random.default_rng(2024)
+    offs = rng.uniform(-2.0, 2.0, D) * np.exp2(rng.integers(0, 11, D))
+    x = rng.standard_normal((N, D)) + offs[None, :]
+    kb = bf16_bits_round(x.astype(np.float32))                     # [N, D] BF16 bits
+    xf = synth.bf16_to_float(kb).astype(np.float64)
+    km = oracle.k_mean(kb[None, :, None, :], plant)[0, 0]
+    shift = 48                                                     # every value is a multiple of 2^-48
+    scaled = xf * 2.0 ** shift
+    assert np.all(scaled == np.round(scaled)) and np.abs(scaled).max() < 2.0 ** 62
+    ints = scaled.astype(np.int64)
+    hi, lo = ints >> 31, ints & ((1 << 31) - 1)                   # both column sums fit in int64
+    sums = [(int(a) << 31) + int(b) for a, b in zip(hi.sum(axis=0), lo.sum(axis=0))]
+    want = np.array([f32_nearest(Fraction(int(s), N << shift)) for s in sums], np.float32)
+    bad = np.flatnonzero(km.view(np.uint32) != want.view(np.uint32))
+    assert bad.size == 0, (bad[:4].tolist(), km[bad[:4]].tolist(), want[bad[:4]].tolist())
+
+
 ALL_PINS = [pin_e4m3_decode, pin_e4m3_encode, pin_f16_round, pin_bf16_round, pin_worked_example,
             pin_group_boundaries, pin_q_zero_mean, pin_fp64_bruteforce, pin_dominance,
             pin_k_offset_invariance, pin_denominator, pin_qk_s32, pin_norm_rope_fp64,
-            pin_norm_rope_exact, pin_int8_ties, pin_f16_slice_buffers, pin_online_rescale_exact]
+            pin_norm_rope_exact, pin_int8_ties, pin_f16_slice_buffers, pin_online_rescale_exact,
+            pin_k_mean_exact]

@@ -24,6 +24,7 @@ PLANTS = {
     16: "Q scale read per 64 rows in the score scale",
     17: "accumulator rescaled after the tile's PV instead of before",
     18: "accumulator not rescaled (the denominator is)",
+    19: "K channel sums kept in FP32",
 }
 
 

@@ -91,7 +91,7 @@ def lib():
             "sage_strerror": [I],
             "sage_set_mainloop": [I],
             "sage_get_mainloop": [],
-            "sage_debug_qk_s32": [P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
+            "sage_debug_qk_s32": [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
             "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
             "sage_debug_set_stall": [I, ctypes.c_longlong],
             "sage_attn_fwd_host": [V, V, V, V, V, V, P, P, L64, L64, L64, I, I, I, I, ctypes.c_float, I, P, SZ,
@@ -288,9 +288,10 @@ def sage_debug_set_stall(k_tile: int, wait_limit_cycles: int = 0):
     _check(lib().sage_debug_set_stall(int(k_tile), int(wait_limit_cycles)), "sage_debug_set_stall")
 
 
-def sage_debug_qk_s32(q_i8, k_i8, B, N, H, D, b, h, q_tile, k_tile, s_out, workspace, stream=None):
-    _check(lib().sage_debug_qk_s32(_ptr(q_i8), _ptr(k_i8), B, N, H, D, b, h, q_tile, k_tile,
-                                   _ptr(s_out), _ptr(workspace),
+def sage_debug_qk_s32(q_i8, q_scale, k_i8, k_scale, v_fp8, v_scale, B, N, H, D, b, h, q_tile, k_tile, s_out,
+                      workspace, stream=None):
+    _check(lib().sage_debug_qk_s32(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_fp8),
+                                   _ptr(v_scale), B, N, H, D, b, h, q_tile, k_tile, _ptr(s_out), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "sage_debug_qk_s32")
 

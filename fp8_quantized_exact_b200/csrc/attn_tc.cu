@@ -101,14 +101,20 @@ __device__ __forceinline__ TcSmem<D>& tc_smem() {
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D>
+// DBG (the score export sage_debug_qk_s32): a one-CTA launch for query tile
+// p.dbg_qt of head (p.dbg_b, p.dbg_h) that runs the whole mainloop and also
+// copies the int32 scores of key tile p.dbg_tile, as its softmax owners read
+// them from TMEM, to p.dbg_out (128 x 64, row-major); it stores no output.
+template <int D, bool DBG>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr int DH = D / 2;  // output columns owned by one output thread
   TcSmem<D>& sm = tc_smem<D>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qt = DBG ? p.dbg_qt : (int)blockIdx.x;
+  const int h = DBG ? p.dbg_h : (int)blockIdx.y;
+  const int b = DBG ? p.dbg_b : (int)blockIdx.z;
   const int bh = b * p.H + h;
   const int T = p.T64;            // 64-key tiles
   const int G = (T + 1) >> 1;     // 128-key groups
@@ -167,6 +173,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       uint32_t S[64];
       tmem_ld64(lane_addr + cols, S);
       tmem_wait_ld();
+      if (DBG && t == p.dbg_tile) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) p.dbg_out[i * kKTile + j] = (int32_t)S[j];
+      }
       // test the handoffs of this tile early; their latency overlaps the max pass
       const bool m_ready = t == 0 || mbar_try(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1));
       const bool r_ready = mbar_try(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1));
@@ -278,7 +288,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
       }
     }
-    if (ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) && !*abort_flag) {
+    if (!DBG && ok && wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) && !*abort_flag) {
       const int row = qt * kQTile + i;
       const float rc = sm.rcp[i];
       if (row < p.N) {
@@ -401,66 +411,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   if (warp == kQkWarp) tmem_free(tmem, kTmemCols);
 }
 
-// ------------------------------------------------ debug: one score tile
-template <int D>
-__global__ void __launch_bounds__(kThreadsTC, 1)
-    debug_qk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const AttnParams p, int b, int h, int qt, int kt, int32_t* s_out) {
-  TcSmem<D>& sm = tc_smem<D>();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = b * p.H + h;
-  volatile int* abort_flag = &sm.abort_flag;
-  if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.kv_full[0], 1);
-    mbar_init(&sm.s_full[0], 1);
-    sm.abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == kQkWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  if (warp == kLoadWarp && lane == 0) {
-    mbar_expect_tx(&sm.q_full, kQTile * D);
-    tma_load_3d(sm.q, &tm_q, 0, qt * kQTile, bh, &sm.q_full);
-    mbar_expect_tx(&sm.kv_full[0], kGroup * D);  // a full stage box; its first 64 keys are the tile
-    tma_load_3d(sm.k[0], &tm_k, 0, kt * kKTile, bh, &sm.kv_full[0]);
-    wait_bounded(&sm.q_full, 0, abort_flag, nullptr, 7, p.wait_limit, false);
-    wait_bounded(&sm.kv_full[0], 0, abort_flag, nullptr, 8, p.wait_limit, false);
-  } else if (warp == kQkWarp) {
-    if (lane == 0) {
-      bool ok = wait_bounded(&sm.q_full, 0, abort_flag, p.status, 9, p.wait_limit) &&
-                wait_bounded(&sm.kv_full[0], 0, abort_flag, p.status, 10, p.wait_limit);
-      if (ok) {
-        tc_fence_after();
-        const uint64_t qdesc = smem_desc(sm.q, D), kdesc = smem_desc(sm.k[0], D);
-#pragma unroll
-        for (int kk = 0; kk < D / 32; ++kk)
-          mma_i8_ss(tmem + kColS, qdesc + 2 * kk, kdesc + 2 * kk, idesc_qk(kKTile), kk > 0);
-      }
-      tc_commit(&sm.s_full[0]);
-      wait_bounded(&sm.s_full[0], 0, abort_flag, nullptr, 14, p.wait_limit, false);
-    }
-    __syncwarp();
-  } else if (warp >= kSoftWarp0 && warp < kSoftWarp0 + 4) {
-    if (wait_bounded(&sm.s_full[0], 0, abort_flag, p.status, 1, p.wait_limit) && !*abort_flag) {
-      tc_fence_after();
-      const int quad = warp & 3;
-      uint32_t S[64];
-      tmem_ld64(tmem + ((uint32_t)(quad * 32) << 16) + kColS, S);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 64; ++j) s_out[(quad * 32 + lane) * kKTile + j] = (int32_t)S[j];
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == kQkWarp) tmem_free(tmem, kTmemCols);
-}
-
 // ------------------------------------------------------------------- host
 template <int D>
 size_t smem_bytes() {
@@ -470,7 +420,7 @@ size_t smem_bytes() {
   return need > 120 * 1024 ? need : 120 * 1024;
 }
 
-template <int D>
+template <int D, bool DBG>
 int launch_tc(const AttnParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const uint64_t bh = (uint64_t)p.B * p.H;
@@ -478,26 +428,12 @@ int launch_tc(const AttnParams& p, cudaStream_t s) {
       !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kGroup) ||
       !make_map(&mv, p.v8, p.Nk, D, bh, p.Nk, (uint64_t)D * p.Nk, kGroup, D))
     return SAGE_ERR_CUDA;
-  auto* fn = attn_tc_kernel<D>;
+  auto* fn = attn_tc_kernel<D, DBG>;
   const size_t smem = smem_bytes<D>();
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  fn<<<dim3(p.Nq / kQTile, p.H, p.B), kThreadsTC, smem, s>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
-}
-
-template <int D>
-int launch_dbg_tc(const AttnParams& p, int b, int h, int qt, int kt, int32_t* s_out, cudaStream_t s) {
-  CUtensorMap mq, mk;
-  const uint64_t bh = (uint64_t)p.B * p.H;
-  if (!make_map(&mq, p.q8, D, p.Nq, bh, D, (uint64_t)p.Nq * D, D, kQTile) ||
-      !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kGroup))
-    return SAGE_ERR_CUDA;
-  auto* fn = debug_qk_tc_kernel<D>;
-  const size_t smem = smem_bytes<D>();
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return SAGE_ERR_CUDA;
-  fn<<<1, kThreadsTC, smem, s>>>(mq, mk, p, b, h, qt, kt, s_out);
+  const dim3 grid = DBG ? dim3(1, 1, 1) : dim3(p.Nq / kQTile, p.H, p.B);
+  fn<<<grid, kThreadsTC, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
@@ -511,15 +447,8 @@ bool tc_available() {
 }
 
 int launch_attn_tc(const AttnParams& p, cudaStream_t s) {
-  if (p.D == 128) return launch_tc<128>(p, s);
-  if (p.D == 64) return launch_tc<64>(p, s);
-  return SAGE_ERR_UNSUPPORTED;
-}
-
-int launch_debug_qk_tc(const AttnParams& p, int b, int h, int q_tile, int k_tile, int32_t* s_out,
-                       cudaStream_t s) {
-  if (p.D == 128) return launch_dbg_tc<128>(p, b, h, q_tile, k_tile, s_out, s);
-  if (p.D == 64) return launch_dbg_tc<64>(p, b, h, q_tile, k_tile, s_out, s);
+  if (p.D == 128) return p.dbg_out ? launch_tc<128, true>(p, s) : launch_tc<128, false>(p, s);
+  if (p.D == 64) return p.dbg_out ? launch_tc<64, true>(p, s) : launch_tc<64, false>(p, s);
   return SAGE_ERR_UNSUPPORTED;
 }
 

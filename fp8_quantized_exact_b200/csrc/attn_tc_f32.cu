@@ -92,13 +92,18 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
   for (int c = 0; c < 64; c += 16) tmem_st16(taddr + c, *reinterpret_cast<const uint32_t(*)[16]>(&r[c]));
 }
 
-template <int D>
+// DBG: the score export of sage_debug_qk_s32, as in the exact mainloop (a
+// one-CTA launch for p.dbg_qt/dbg_h/dbg_b that copies the int32 scores of key
+// tile p.dbg_tile to p.dbg_out and stores no output).
+template <int D, bool DBG>
 __global__ void __launch_bounds__(kThreadsF, 1)
     attn_tc_f32_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   F32Smem<D>& sm = f32_smem<D>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qt = DBG ? p.dbg_qt : (int)blockIdx.x;
+  const int h = DBG ? p.dbg_h : (int)blockIdx.y;
+  const int b = DBG ? p.dbg_b : (int)blockIdx.z;
   const int bh = b * p.H + h;
   const int T = p.T64;
   const int G = (T + 1) >> 1;
@@ -155,6 +160,10 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       uint32_t S[64];
       tmem_ld64(lane_addr + cols, S);
       tmem_wait_ld();
+      if (DBG && t == p.dbg_tile) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) p.dbg_out[i * kKTile + j] = (int32_t)S[j];
+      }
       const bool m_ready = t == 0 || __all_sync(0xffffffffu, mbar_try(&sm.m_full[quad][par ^ 1], (uint32_t)(((t - 1) >> 1) & 1)));
       const bool r_ready = __all_sync(0xffffffffu, mbar_try(&sm.r_free[par], (uint32_t)(((t >> 1) & 1) ^ 1)));
       const float cs = __fmul_rn(__fmul_rn(qs, ks), p.sl2);
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(kThreadsF, 1)
       mbar_arrive(&sm.c_done);
     }
     // epilogue: the last PV MMAs have completed and 1/d is known
-    if (ok && T > 0 &&
+    if (!DBG && ok && T > 0 &&
         wait_bounded(&sm.o_acc[(T - 1) & 3], (uint32_t)(((T - 1) >> 2) & 1), abort_flag, p.status, 21, p.wait_limit) &&
         wait_bounded(&sm.done, 0, abort_flag, p.status, 5, p.wait_limit) && !*abort_flag) {
       tc_fence_after();
@@ -387,7 +396,7 @@ size_t f32_smem_bytes() {
   return need > 120 * 1024 ? need : 120 * 1024;  // one CTA (and one 512-column TMEM request) per SM
 }
 
-template <int D>
+template <int D, bool DBG>
 int launch_f32(const AttnParams& p, cudaStream_t s) {
   CUtensorMap mq, mk, mv;
   const uint64_t bh = (uint64_t)p.B * p.H;
@@ -395,19 +404,20 @@ int launch_f32(const AttnParams& p, cudaStream_t s) {
       !make_map(&mk, p.k8, D, p.Nk, bh, D, (uint64_t)p.Nk * D, D, kGroupF) ||
       !make_map(&mv, p.v8, p.Nk, D, bh, p.Nk, (uint64_t)D * p.Nk, kGroupF, D))
     return SAGE_ERR_CUDA;
-  auto* fn = attn_tc_f32_kernel<D>;
+  auto* fn = attn_tc_f32_kernel<D, DBG>;
   const size_t smem = f32_smem_bytes<D>();
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  fn<<<dim3(p.Nq / kQTile, p.H, p.B), kThreadsF, smem, s>>>(mq, mk, mv, p);
+  const dim3 grid = DBG ? dim3(1, 1, 1) : dim3(p.Nq / kQTile, p.H, p.B);
+  fn<<<grid, kThreadsF, smem, s>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 }  // namespace
 
 int launch_attn_tc_f32(const AttnParams& p, cudaStream_t s) {
-  if (p.D == 128) return launch_f32<128>(p, s);
-  if (p.D == 64) return launch_f32<64>(p, s);
+  if (p.D == 128) return p.dbg_out ? launch_f32<128, true>(p, s) : launch_f32<128, false>(p, s);
+  if (p.D == 64) return p.dbg_out ? launch_f32<64, true>(p, s) : launch_f32<64, false>(p, s);
   return SAGE_ERR_UNSUPPORTED;
 }
 

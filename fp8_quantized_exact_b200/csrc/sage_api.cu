@@ -167,6 +167,9 @@ AttnParams make_params(const Dims& d, const int8_t* q8, const float* qs, const i
   p.status = static_cast<DeviceStatus*>(status);
   p.wait_limit = g_wait_limit.load();
   p.stall_tile = g_stall_tile.load();
+  p.dbg_qt = p.dbg_h = p.dbg_b = 0;
+  p.dbg_tile = -1;
+  p.dbg_out = nullptr;
   return p;
 }
 
@@ -531,25 +534,38 @@ int sage_debug_set_stall(int k_tile, long long wait_limit_cycles) {
   return SAGE_OK;
 }
 
-int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int H, int D, int b,
-                      int h, int q_tile, int k_tile, int32_t* s_out, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+int sage_debug_qk_s32(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                      const uint8_t* v_fp8, const float* v_scale, int B, int N, int H, int D, int b, int h,
+                      int q_tile, int k_tile, int32_t* s_out, void* workspace, size_t workspace_bytes,
+                      void* stream) {
   int rc = check_dims(B, N, H, D);
   if (rc) return rc;
   const Dims d = make_dims(B, N, H, D);
-  if (!q_i8 || !k_i8 || !s_out || empty(B, N, H)) return SAGE_ERR_INVALID_ARG;
+  if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v_fp8 || !v_scale || !s_out || empty(B, N, H))
+    return SAGE_ERR_INVALID_ARG;
   if (b < 0 || b >= B || h < 0 || h >= H || q_tile < 0 || q_tile >= d.Nq / kQTile || k_tile < 0 ||
       k_tile >= d.T64)
     return SAGE_ERR_INVALID_ARG;
-  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(s_out)) return SAGE_ERR_UNSUPPORTED;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v_fp8) || !aligned16(q_scale) || !aligned16(k_scale) ||
+      !aligned16(v_scale) || !aligned16(s_out))
+    return SAGE_ERR_UNSUPPORTED;
   if ((rc = check_ws(workspace, workspace_bytes, plan(SAGE_OP_DEBUG_QK, d).total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
-  AttnParams p = make_params(d, q_i8, nullptr, k_i8, nullptr, nullptr, nullptr, nullptr, 0, 0, 0,
-                             0.0f, workspace);
-  return resolved_mainloop() != SAGE_MAINLOOP_MMA_SYNC  // both tcgen05 variants share the QK
-             ? launch_debug_qk_tc(p, b, h, q_tile, k_tile, s_out, s)
-             : launch_debug_qk_mma(p, b, h, q_tile, k_tile, s_out, s);
+  AttnParams p = make_params(d, q_i8, q_scale, k_i8, k_scale, v_fp8, v_scale, nullptr, 0, 0, 0, 0.0f, workspace);
+  switch (resolved_mainloop()) {
+    case SAGE_MAINLOOP_TCGEN05:
+    case SAGE_MAINLOOP_TCGEN05_F32:
+      // one CTA of the mainloop itself, which copies the scores it reads
+      p.dbg_qt = q_tile;
+      p.dbg_h = h;
+      p.dbg_b = b;
+      p.dbg_tile = k_tile;
+      p.dbg_out = s_out;
+      return run_mainloop(p, s);
+    default:
+      return launch_debug_qk_mma(p, b, h, q_tile, k_tile, s_out, s);
+  }
 }
 
 }  // extern "C"

@@ -37,6 +37,11 @@ struct AttnParams {
   DeviceStatus* status;
   long long wait_limit;  // clock cycles a bounded device wait may spin
   int stall_tile;        // test hook: the producer withholds this K/V tile (-1: none)
+  // score export of the mainloop's own QK path (sage_debug_qk_s32): the CTA
+  // of query tile dbg_qt of head (dbg_b, dbg_h) copies the int32 scores of
+  // key tile dbg_tile to dbg_out (128 x 64, row-major)
+  int dbg_qt, dbg_h, dbg_b, dbg_tile;
+  int32_t* dbg_out;
 };
 
 constexpr long long kDefaultWaitLimit = 2000000000LL;  // ~1 s at 1.9 GHz
@@ -144,7 +149,5 @@ int launch_debug_qk_mma(const AttnParams& p, int b, int h, int q_tile, int k_til
                         cudaStream_t s);
 int launch_attn_tc(const AttnParams& p, cudaStream_t s);
 int launch_attn_tc_f32(const AttnParams& p, cudaStream_t s);
-int launch_debug_qk_tc(const AttnParams& p, int b, int h, int q_tile, int k_tile, int32_t* s_out,
-                       cudaStream_t s);
 bool tc_available();
 }  // namespace sage

@@ -196,8 +196,6 @@ __device__ __forceinline__ void tmem_free(uint32_t base, uint32_t cols) {
 
 
 // ------------------------------------------------------------- softmax helpers
-constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: float bits of (magic + S) are magic_bits + S
-
 // Tile maximum fl32(max(S) * c) of one row's 64 scores (the max of the
 // integers is exact, and rounding is monotone with c >= 0); TAIL masks keys
 // >= nvalid.
@@ -218,10 +216,14 @@ __device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int
 }
 
 // Probabilities of 16 of a row's keys (k0..k0+15) against the running max:
-// p = 2^(s - m_new) in FP32 into the partial sums rs, E4M3 bytes (key order
-// from the low byte) into P[k0/4 ..].  nkofs = -(magic*c + m_new), rounded once.
+// p = 2^(fl32(S*c - m_new)) in FP32 into the partial sums rs, E4M3 bytes (key
+// order from the low byte) into P[k0/4 ..].  The exponent argument is one
+// fused multiply-add on the exact float of S (|S| < 2^22, so the conversion
+// is exact).  Scalar operations and this statement order measured fastest of
+// the exact forms tried (packed FP32x2 pairs, a float image with a packed or
+// scalar unbias).
 template <bool TAIL>
-__device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, float cs, float nkofs, int nvalid,
+__device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, float cs, float nm, int nvalid,
                                           float (&rs)[4], uint32_t (&P)[16]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -229,27 +231,17 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, floa
 #pragma unroll
     for (int e = 0; e < 4; e += 2) {
       const int j = 4 * q + e;
-      // exponent arguments fl32(fb*c - kofs) on the exact float images
-      // fb = magic + S, two per packed FMA
-      const float f0 = __int_as_float((int32_t)Sc[j] + 0x4B400000);
-      const float f1 = __int_as_float((int32_t)Sc[j + 1] + 0x4B400000);
-      asm("{.reg .b64 x, c, o; mov.b64 x, {%2, %3}; mov.b64 c, {%4, %4}; mov.b64 o, {%5, %5};"
-          " fma.rn.f32x2 x, x, c, o; mov.b64 {%0, %1}, x;}"
-          : "=f"(pv[e]), "=f"(pv[e + 1])
-          : "f"(f0), "f"(f1), "f"(cs), "f"(nkofs));
+      pv[e] = __fmaf_rn(__int2float_rn((int32_t)Sc[j]), cs, nm);
+      pv[e + 1] = __fmaf_rn(__int2float_rn((int32_t)Sc[j + 1]), cs, nm);
       pv[e] = ex2(pv[e]);
       pv[e + 1] = ex2(pv[e + 1]);
       if (TAIL && k0 + j >= nvalid) pv[e] = 0.0f;
       if (TAIL && k0 + j + 1 >= nvalid) pv[e + 1] = 0.0f;
     }
-    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
-        " mov.b64 {%0, %1}, a;}"
-        : "+f"(rs[0]), "+f"(rs[1])
-        : "f"(pv[0]), "f"(pv[1]));
-    asm("{.reg .b64 a, b; mov.b64 a, {%0, %1}; mov.b64 b, {%2, %3}; add.rn.f32x2 a, a, b;"
-        " mov.b64 {%0, %1}, a;}"
-        : "+f"(rs[2]), "+f"(rs[3])
-        : "f"(pv[2]), "f"(pv[3]));
+    rs[0] = __fadd_rn(rs[0], pv[0]);
+    rs[1] = __fadd_rn(rs[1], pv[1]);
+    rs[2] = __fadd_rn(rs[2], pv[2]);
+    rs[3] = __fadd_rn(rs[3], pv[3]);
     asm("{.reg .b16 lo, hi; cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1; cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;"
         " mov.b32 %0, {lo, hi};}"
         : "=r"(P[k0 / 4 + q])
@@ -262,21 +254,21 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, floa
 // pass are free.  Returns the FP32 row sum.
 template <bool TAIL>
 __device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new, int nvalid, uint32_t (&P)[16]) {
-  const float nkofs = -__fmaf_rn(kMagic, cs, m_new);
+  const float nm = -m_new;
   float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   uint32_t A[16], Bc[16];
   tmem_ld16(taddr, A);
   tmem_wait_ld16(A);
   tmem_ld16(taddr + 16, Bc);
-  chunk_exp<TAIL>(A, 0, cs, nkofs, nvalid, rs, P);
+  chunk_exp<TAIL>(A, 0, cs, nm, nvalid, rs, P);
   tmem_wait_ld16(Bc);
   tmem_ld16(taddr + 32, A);
-  chunk_exp<TAIL>(Bc, 16, cs, nkofs, nvalid, rs, P);
+  chunk_exp<TAIL>(Bc, 16, cs, nm, nvalid, rs, P);
   tmem_wait_ld16(A);
   tmem_ld16(taddr + 48, Bc);
-  chunk_exp<TAIL>(A, 32, cs, nkofs, nvalid, rs, P);
+  chunk_exp<TAIL>(A, 32, cs, nm, nvalid, rs, P);
   tmem_wait_ld16(Bc);
-  chunk_exp<TAIL>(Bc, 48, cs, nkofs, nvalid, rs, P);
+  chunk_exp<TAIL>(Bc, 48, cs, nm, nvalid, rs, P);
   return __fadd_rn(__fadd_rn(rs[0], rs[1]), __fadd_rn(rs[2], rs[3]));
 }
 

@@ -310,12 +310,27 @@ SAGE_API int sage_attn_fwd_noalloc(sage_view_bf16 q, sage_view_bf16 k, sage_view
                                    int64_t out_stride_h, int B, int N, int H, int D,
                                    float sm_scale, void* stream);
 
-/* Test export: the int32 Q K^T tile that the selected mainloop computes for
- * query tile q_tile (128 rows) and key tile k_tile (64 keys) of head (b, h),
- * written to s_out[128][64] (device, row-major, natural key order). */
-SAGE_API int sage_debug_qk_s32(const int8_t* q_i8, const int8_t* k_i8, int B, int N, int H, int D, int b,
-                      int h, int q_tile, int k_tile, int32_t* s_out, void* workspace,
-                      size_t workspace_bytes, void* stream);
+/* Test export: the int32 Q K^T scores of query tile q_tile (128 rows) and
+ * key tile k_tile (64 keys) of head (b, h), written to s_out[128][64]
+ * (device, row-major, natural key order).  The operation is the per-tile
+ * INT8 QK^T of "State-Ownership Architecture Decision", section
+ * "Non-Negotiable Dataflow".
+ *   - With a tcgen05 mainloop selected, the scores come from the mainloop
+ *     itself: one CTA of it runs for (b, h, q_tile) over all key tiles, with
+ *     the same TMA ring, descriptors and 128-key MMAs as a forward call, and
+ *     copies the tile's scores as its softmax owners read them from tensor
+ *     memory.  It stores no attention output.
+ *   - With the mma.sync mainloop, a one-tile kernel runs that mainloop's
+ *     fragment code for the QK product.
+ * The quantised tensors are those sage_quant_qk / sage_quant_v produce (the
+ * scales and V are read by the mainloop run).  workspace: at least
+ * sage_workspace_bytes(SAGE_OP_DEBUG_QK, ...).  Errors as for
+ * sage_attn_from_quant, and SAGE_ERR_INVALID_ARG for an out-of-range
+ * (b, h, q_tile, k_tile). */
+SAGE_API int sage_debug_qk_s32(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8, const float* k_scale,
+                               const uint8_t* v_fp8, const float* v_scale, int B, int N, int H, int D, int b, int h,
+                               int q_tile, int k_tile, int32_t* s_out, void* workspace, size_t workspace_bytes,
+                               void* stream);
 
 #ifdef __cplusplus
 }

@@ -7,6 +7,19 @@ import numpy as np
 
 TOL_MAX_ABS = 2e-2   # output tolerance: max |gpu - oracle| over all compared elements
 TOL_MEAN_ABS = 1e-3  # and the mean of |gpu - oracle|
+# per-head ||gpu - oracle|| / ||oracle|| on the sampled rows of the full-size
+# workloads: the GPU and the oracle round the same operations in the same
+# order except the exponential (ex2.approx against a correctly rounded exp2,
+# a few ulp) and the single rounding of the exponent argument; those flip
+# isolated E4M3 probability codes, each moving an output by a fraction of one
+# key's weight.  1e-3 is far below the error of the quantisation itself
+# (several percent) yet above what such flips can add up to (measured: at
+# most 1.2e-4 for the tcgen05 mainloop).  The legacy mma.sync mainloop's FP16
+# accumulator rounds inside each 32-term slice sum instead of once (see
+# tests/test_gpu_golden.py), which moves outputs further (measured: up to
+# 1.15e-3): its bound is 3e-3.
+TOL_REL_L2 = 1e-3
+TOL_REL_L2_MMA_SYNC = 3e-3
 
 
 def to_device(inp, dev):

@@ -113,7 +113,15 @@ def test_argument_errors_need_no_device(lib):
         assert lib.sage_set_mainloop(which) == sage.SAGE_OK
         assert lib.sage_get_mainloop() == which
     assert lib.sage_set_mainloop(sage.SAGE_MAINLOOP_DEFAULT) == sage.SAGE_OK
-    assert lib.sage_debug_qk_s32(4096, 4096, 1, 100, 2, 64, 0, 2, 0, 0, 4096, 4096, 4096, None) == sage.SAGE_ERR_INVALID_ARG
+    dbg = lib.sage_debug_qk_s32
+    assert dbg(4096, 4096, 4096, 4096, 4096, 4096, 1, 100, 2, 64, 0, 2, 0, 0, 4096, 4096, 4096,
+               None) == sage.SAGE_ERR_INVALID_ARG                     # head 2 of 2
+    assert dbg(4096, 4096, 4096, 4096, 4096, 4096, 1, 100, 2, 64, 0, 1, 1, 0, 4096, 4096, 4096,
+               None) == sage.SAGE_ERR_INVALID_ARG                     # query tile 1 of 1
+    assert dbg(4096, 4096, 4096, 4096, 4096, 4096, 1, 100, 2, 64, 0, 1, 0, 2, 4096, 4096, 4096,
+               None) == sage.SAGE_ERR_INVALID_ARG                     # key tile 2 of 2
+    assert dbg(4096, None, 4096, 4096, 4096, 4096, 1, 100, 2, 64, 0, 1, 0, 0, 4096, 4096, 4096,
+               None) == sage.SAGE_ERR_INVALID_ARG                     # missing scale
     host = lib.sage_attn_fwd_host
     other = sage.sage_view_bf16(8192, 256 * 2 * 128, 2 * 128, 128)
     narrow = sage.sage_view_bf16(4096, 256 * 2 * 128, 32, 128)

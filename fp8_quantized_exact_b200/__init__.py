@@ -44,7 +44,7 @@ EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_
            "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
            "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
-           "sage_attn_fwd_noalloc", "sage_debug_set_stall", "sage_attn_fwd_host")
+           "sage_attn_fwd_noalloc", "sage_noalloc_read_status", "sage_debug_set_stall", "sage_attn_fwd_host")
 SAGE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -93,6 +93,7 @@ def lib():
             "sage_get_mainloop": [],
             "sage_debug_qk_s32": [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, P, SZ, P],
             "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
+            "sage_noalloc_read_status": [P],
             "sage_debug_set_stall": [I, ctypes.c_longlong],
             "sage_attn_fwd_host": [V, V, V, V, V, V, P, P, L64, L64, L64, I, I, I, I, ctypes.c_float, I, P, SZ,
                                    P, P, P, P, P, P, P],
@@ -217,6 +218,12 @@ def sage_attn_fwd_noalloc(q, k, v, out, sm_scale, stream=None):
                                        out.stride(1), out.stride(2), B, N, H, D, float(sm_scale),
                                        _stream(stream)),
            "sage_attn_fwd_noalloc")
+
+
+def sage_noalloc_read_status(stream=None) -> int:
+    """Wait for the stream and return the status code of the last no-alloc
+    call on the current device (SAGE_OK, SAGE_ERR_TIMEOUT, ...)."""
+    return int(lib().sage_noalloc_read_status(_stream(stream)))
 
 
 def _host_view(t) -> sage_view_bf16:

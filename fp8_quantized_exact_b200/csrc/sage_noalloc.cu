@@ -62,3 +62,12 @@ extern "C" SAGE_API int sage_attn_fwd_noalloc(sage_view_bf16 q, sage_view_bf16 k
   return sage_attn_fwd(q, k, v, out, out_stride_b, out_stride_n, out_stride_h, B, N, H, D,
                        sm_scale, scratch, (size_t)SAGE_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// The status word at the start of the fixed array (sage_attn_fwd clears it
+// at the start of each call and the kernels record their errors there).
+extern "C" SAGE_API int sage_noalloc_read_status(void* stream) {
+  void* scratch = nullptr;
+  const int rc = scratch_address(&scratch);
+  if (rc != SAGE_OK) return rc;
+  return sage_read_device_status(scratch, stream);
+}

@@ -310,6 +310,18 @@ SAGE_API int sage_attn_fwd_noalloc(sage_view_bf16 q, sage_view_bf16 k, sage_view
                                    int64_t out_stride_h, int B, int N, int H, int D,
                                    float sm_scale, void* stream);
 
+/* The device status of the last sage_attn_fwd_noalloc call on the current
+ * device (no counterpart in the pages: it reads the status word that the
+ * fixed array holds in place of a workspace's).  A caller of the no-alloc
+ * entry point has no workspace to pass to sage_read_device_status; this call
+ * does the same for the array: it waits for `stream` (the host blocks until
+ * the work queued there is done) and returns SAGE_OK or the code a kernel
+ * recorded, e.g. SAGE_ERR_TIMEOUT when a bounded wait ran out and the output
+ * was left partly written.  SAGE_ERR_CUDA if the copy or the wait fails.  The
+ * word belongs to whichever call last cleared it: read it before the next
+ * no-alloc call on the device. */
+SAGE_API int sage_noalloc_read_status(void* stream);
+
 /* Test export: the int32 Q K^T scores of query tile q_tile (128 rows) and
  * key tile k_tile (64 keys) of head (b, h), written to s_out[128][64]
  * (device, row-major, natural key order).  The operation is the per-tile

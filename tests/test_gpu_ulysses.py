@@ -1,7 +1,9 @@
 """Ulysses wrapper on one GPU: a one-rank NCCL group runs the real exchanges
-and the library's attention on the strided head-shard views; the output
-must equal a direct sage_attn_fwd call bit for bit (the exchange is a pure
-relayout).  Several ranks are covered by the two-rank CPU test."""
+and the library's attention on the strided head-shard views.  The output is
+checked against the CPU oracle's attention on the same inputs (within the
+output tolerance), and against a direct sage_attn_fwd call bit for bit (the
+exchange is a pure relayout).  Several ranks are covered by the two- and
+four-rank CPU tests."""
 import datetime
 import os
 import socket
@@ -9,6 +11,7 @@ import socket
 import pytest
 
 import gpu_util as gu
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -52,4 +55,7 @@ def test_one_rank_ulysses_equals_direct_call(sage, shape, layout):
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+    qz = oracle.quantize(inp.q, inp.k, inp.v)
+    want = oracle.bf16_bits_to_float(oracle.attention(qz))
+    gu.compare_out(out.float().cpu().numpy(), want, f"ulysses {shape} {layout}")
     assert torch.equal(out.view(torch.int16), ref.view(torch.int16))

@@ -222,6 +222,20 @@ def whole_job_tops(ops_per_rank: float, world: int, ms_per_step: float) -> float
 
 
 # --------------------------------------------------------------- reference
+def host_cpu():
+    """The host's CPU model (from /proc/cpuinfo) and its logical CPU count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 def cpu_sample(cfg, inp, groups: int):
     """Time the oracle on a bounded sample of the workload and extrapolate the
     whole-workload time: the full prepass of two heads (scaled by B*H/2) and
@@ -246,7 +260,8 @@ def cpu_sample(cfg, inp, groups: int):
             rows += n
     bh = cfg.B * cfg.H
     total_s = t_pre * bh / len(heads) + t_att * (bh * cfg.N) / rows
-    return {"value": cfg.ops / total_s / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle",
+    return {"value": cfg.ops / total_s / 1e12, "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
+            "extrapolated": True,
             "sample": f"full prepass of {len(heads)} heads + attention of {rows} query rows "
                       f"({len(gl)} 32-row groups x {len(heads)} heads) of {cfg.name}; "
                       f"extrapolated to all B*H heads and N rows",
@@ -278,9 +293,11 @@ def run_reference(args, cfg, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64 (CPU)",
             "data": "synthetic (seeded normal BF16 stand-in for the pages' video-DiT activations)",
-            "config": {"workload": f"{cfg.name}: {cfg.about}"},
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": vals[0]["sample"]},
+            "config": {"workload": f"{cfg.name}: {cfg.about}", "B": cfg.B, "N": cfg.N, "H": cfg.H,
+                       "D": cfg.D},
+            "extrapolated": True,
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", **host_cpu(),
+                             "sample": vals[0]["sample"], "extrapolated": True},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "wall_s": round(wall, 1)}
     print(json.dumps(line), flush=True)

@@ -267,20 +267,16 @@ def test_long_context_tile_geometry(lib):
     assert lay["v_scale"] - lay["v_fp8"] >= 56 * 128 * 591 * 64
 
 
-def test_readme_c_example_compiles(lib, tmp_path):
-    """The C example in README.md compiles as C11 against the header and the
-    CUDA runtime header, and links against the library and cudart (it needs
-    a GPU only to run)."""
+def test_c_example_compiles(lib, tmp_path):
+    """The C example (tests/c_example/attend.c, the code README.md shows)
+    compiles as C11 against the header and the CUDA runtime header, and links
+    against the library and cudart (it needs a GPU only to run)."""
     import shutil
     import subprocess
     gcc, cuda_inc = shutil.which("gcc"), "/usr/local/cuda/include"
     if gcc is None or not os.path.isdir(cuda_inc):
         pytest.skip("no C compiler or CUDA headers")
-    with open(os.path.join(ROOT, "README.md")) as f:
-        blocks = re.findall(r"```c\n(.*?)```", f.read(), re.S)
-    assert len(blocks) == 1
-    src = tmp_path / "example.c"
-    src.write_text(blocks[0])
+    src = os.path.join(ROOT, "tests", "c_example", "attend.c")
     obj = tmp_path / "example.o"
     cc = subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I",
                          os.path.join(ROOT, "include"), "-isystem", cuda_inc, "-c", str(src), "-o", str(obj)],

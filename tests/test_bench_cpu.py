@@ -47,6 +47,11 @@ def test_reference_step_size_follows_the_budget(monkeypatch, capsys):
     for key in ("metric", "value", "unit", "ms_per_step", "cpu_baseline", "e2e", "higher_is_better"):
         assert key in line
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # the same workload keys as the GPU arm's line, the host named, the step extrapolated
+    cfg = synth.CONFIGS["small"]
+    assert {k: line["config"][k] for k in "BNHD"} == {"B": cfg.B, "N": cfg.N, "H": cfg.H, "D": cfg.D}
+    assert line["extrapolated"] is True and line["cpu_baseline"]["extrapolated"] is True
+    assert line["cpu_baseline"]["nproc"] == os.cpu_count() and "cpu_model" in line["cpu_baseline"]
 
 
 def test_reference_step_size_is_bounded(monkeypatch, capsys):

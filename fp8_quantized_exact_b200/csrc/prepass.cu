@@ -35,14 +35,13 @@ __device__ __forceinline__ uint32_t i8_code(float x, float inv) {
 }
 
 // ------------------------------------------------------------------------
-// Per 64-token chunk: FP64 sum of each K channel (tokens added in order) and
-// the FP32 amax of each V channel.  One thread owns 8 consecutive channels
-// of one chunk; D/8 threads per chunk; 128 threads per block.
-template <int D, bool DO_K, bool DO_V>
-__global__ void __launch_bounds__(128) chunk_stats_kernel(
-    const uint16_t* __restrict__ k, int64_t ksb, int64_t ksn, int64_t ksh,
-    const uint16_t* __restrict__ v, int64_t vsb, int64_t vsn, int64_t vsh, int N, int H, int T64,
-    double* __restrict__ k_part, float* __restrict__ v_part) {
+// K: per 64-token chunk, the FP64 sum of each channel (tokens added in
+// order).  One thread owns 8 consecutive channels of one chunk; D/8 threads
+// per chunk; 128 threads per block.
+template <int D>
+__global__ void __launch_bounds__(128, 8) k_sums_kernel(const uint16_t* __restrict__ k, int64_t sb, int64_t sn,
+                                                     int64_t sh, int N, int H, int T64,
+                                                     double* __restrict__ k_part) {
   constexpr int TPC = D / 8;
   constexpr int CPB = 128 / TPC;
   const int chunk = blockIdx.x * CPB + threadIdx.x / TPC;
@@ -52,102 +51,168 @@ __global__ void __launch_bounds__(128) chunk_stats_kernel(
   const int n0 = chunk * kKTile;
   const int n1 = min(n0 + kKTile, N);
   double ks[8];
-  float vm[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) { ks[i] = 0.0; vm[i] = 0.0f; }
-  const uint16_t* kp = k + b * ksb + h * ksh + col;
-  const uint16_t* vp = v + b * vsb + h * vsh + col;
+  for (int i = 0; i < 8; ++i) ks[i] = 0.0;
+  const uint16_t* kp = k + b * sb + h * sh + col;
 #pragma unroll 4
   for (int n = n0; n < n1; ++n) {
-    if (DO_K) {
-      float f[8];
-      unpack_bf16x8(ldg16(kp + n * ksn), f);
+    float f[8];
+    unpack_bf16x8(ldg16(kp + n * sn), f);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) ks[i] = __dadd_rn(ks[i], (double)f[i]);
+    for (int i = 0; i < 8; ++i) ks[i] = __dadd_rn(ks[i], (double)f[i]);
+  }
+  double2* dst = reinterpret_cast<double2*>(k_part + (((size_t)b * H + h) * T64 + chunk) * D + col);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dst[i] = make_double2(ks[2 * i], ks[2 * i + 1]);
+}
+
+// Chunk partials -> k_mean: the partials added in chunk order, then one FP64
+// division and one rounding to FP32.  One 128-thread block per head; pieces
+// of kKMeanPiece chunks x D partials are copied into shared memory with
+// cp.async (two buffers: the next piece streams in while thread d < D adds
+// channel d of the current one), so the sequential sums run from shared
+// memory instead of waiting on each load.
+constexpr int kKMeanPiece = 32;
+
+template <int D>
+__global__ void __launch_bounds__(128) k_mean_kernel(int N, int T64, const double* __restrict__ k_part,
+                                                     float* __restrict__ k_mean) {
+  extern __shared__ __align__(16) double kbuf[];  // [2][kKMeanPiece][D]
+  const size_t bh = blockIdx.x;
+  const double* src = k_part + bh * T64 * D;
+  const int pieces = ceil_div(T64, kKMeanPiece);
+  auto fetch = [&](int pc) {
+    const int c0 = pc * kKMeanPiece, n = min(kKMeanPiece, T64 - c0);
+    double* dst = kbuf + (pc & 1) * kKMeanPiece * D;
+    for (int i = threadIdx.x; i < n * D / 2; i += 128)  // 16-byte pairs of doubles
+      cp_async_16(smem_u32(dst + 2 * i), src + (size_t)c0 * D + 2 * i);
+    cp_async_commit();
+  };
+  fetch(0);
+  double total = 0.0;
+  for (int pc = 0; pc < pieces; ++pc) {
+    if (pc + 1 < pieces) {
+      fetch(pc + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    if (DO_V) {
+    __syncthreads();
+    const int n = min(kKMeanPiece, T64 - pc * kKMeanPiece);
+    const double* cur = kbuf + (pc & 1) * kKMeanPiece * D;
+    if (threadIdx.x < D)
+      for (int c = 0; c < n; ++c) total = __dadd_rn(total, cur[c * D + threadIdx.x]);
+    __syncthreads();  // the buffer is refilled two pieces on
+  }
+  if (threadIdx.x < D) k_mean[bh * D + threadIdx.x] = __double2float_rn(__ddiv_rn(total, (double)N));
+}
+
+template <int D>
+void launch_k_mean(int BH, int N, int T64, const double* k_part, float* k_mean, cudaStream_t s) {
+  const size_t smem = 2 * kKMeanPiece * D * sizeof(double);  // 64 KB at D = 128
+  cudaFuncSetAttribute(k_mean_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  k_mean_kernel<D><<<BH, 128, smem, s>>>(N, T64, k_part, k_mean);
+}
+
+// V: the FP32 amax of each channel over all tokens.  A block takes 8 * 128/D
+// chunks of 64 tokens, reduces them in shared memory and merges the result
+// into v_amax[b][h][d] (zero at the launch) with an integer atomic max: the
+// amax of non-negative floats is exact in any order, and their bit patterns
+// order as integers.
+template <int D>
+__global__ void __launch_bounds__(128) v_amax_kernel(const uint16_t* __restrict__ v, int64_t sb, int64_t sn,
+                                                     int64_t sh, int N, int H, int T64, float* __restrict__ v_amax) {
+  constexpr int TPC = D / 8;
+  constexpr int CPB = 128 / TPC;
+  __shared__ float red[CPB][D];
+  const int cl = threadIdx.x / TPC;
+  const int chunk = blockIdx.x * CPB + cl;
+  const int col = (threadIdx.x % TPC) * 8;
+  const int h = blockIdx.y, b = blockIdx.z;
+  float vm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) vm[i] = 0.0f;
+  if (chunk < T64) {
+    const int n0 = chunk * kKTile;
+    const int n1 = min(n0 + kKTile, N);
+    const uint16_t* vp = v + b * sb + h * sh + col;
+#pragma unroll 4
+    for (int n = n0; n < n1; ++n) {
       float f[8];
-      unpack_bf16x8(ldg16(vp + n * vsn), f);
+      unpack_bf16x8(ldg16(vp + n * sn), f);
 #pragma unroll
       for (int i = 0; i < 8; ++i) vm[i] = fmaxf(vm[i], fabsf(f[i]));
     }
   }
-  const size_t o = ((size_t)(b * H + h) * T64 + chunk) * D + col;
-  if (DO_K) {
-    double2* dst = reinterpret_cast<double2*>(k_part + o);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_double2(ks[2 * i], ks[2 * i + 1]);
-  }
-  if (DO_V) {
-    float4* dst = reinterpret_cast<float4*>(v_part + o);
-    dst[0] = make_float4(vm[0], vm[1], vm[2], vm[3]);
-    dst[1] = make_float4(vm[4], vm[5], vm[6], vm[7]);
-  }
-}
-
-// Chunk partials -> k_mean (partials added in chunk order, then one FP64
-// division and one rounding to FP32) and V amax / v_scale.  One thread per
-// (b, h, d).
-template <bool DO_K, bool DO_V>
-__global__ void reduce_stats_kernel(int N, int D, int T64, const double* __restrict__ k_part,
-                                    float* __restrict__ k_mean, const float* __restrict__ v_part,
-                                    float* __restrict__ v_scale, float* __restrict__ v_amax) {
-  const int d = threadIdx.x;
-  const size_t bh = blockIdx.x;
-  if (d >= D) return;
-  if (DO_K) {
-    double total = 0.0;
-    for (int c = 0; c < T64; ++c) total = __dadd_rn(total, k_part[(bh * T64 + c) * D + d]);
-    k_mean[bh * D + d] = __double2float_rn(__ddiv_rn(total, (double)N));
-  }
-  if (DO_V) {
-    float am = 0.0f;
-    for (int c = 0; c < T64; ++c) am = fmaxf(am, v_part[(bh * T64 + c) * D + d]);
-    v_amax[bh * D + d] = am;
-    v_scale[bh * D + d] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
+  for (int i = 0; i < 8; ++i) red[cl][col + i] = vm[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float am = red[0][threadIdx.x];
+#pragma unroll
+    for (int c = 1; c < CPB; ++c) am = fmaxf(am, red[c][threadIdx.x]);
+    atomicMax(reinterpret_cast<int*>(v_amax) + ((size_t)b * H + h) * D + threadIdx.x, __float_as_int(am));
   }
 }
 
 // ------------------------------------------------------------------------
-// Q: one warp per 32-row group, four warps per 128-row block (the rows of a
-// block are one mainloop query tile).  Pad rows and pad groups get zeros.
+// Q: one 128-thread block per 64 rows (two 32-row groups, each with its own
+// scale).  Thread t holds 16-byte segments t + 128 i of the 64 x D block in
+// registers between the amax pass and the code pass; its first PER/2
+// segments lie in group 0, the rest in group 1.  Pad rows get zero codes,
+// pad groups no scale.
 template <int D>
-__global__ void __launch_bounds__(128) quant_q_kernel(const uint16_t* __restrict__ q, int64_t sb,
-                                                      int64_t sn, int64_t sh, int N, int H, int Nq,
-                                                      int G32, int8_t* __restrict__ q8,
-                                                      float* __restrict__ q_scale) {
-  constexpr int SEG = D / 8;  // 16-byte segments per row == segments per lane
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = blockIdx.x * 4 + warp;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int r0 = g * kQGroup;
-  uint4 x[SEG];
-  float amax = 0.0f;
+__global__ void __launch_bounds__(128, 6) quant_q_kernel(const uint16_t* __restrict__ q, int64_t sb,
+                                                         int64_t sn, int64_t sh, int N, int H, int Nq,
+                                                         int G32, int8_t* __restrict__ q8,
+                                                         float* __restrict__ q_scale) {
+  constexpr int SEG = D / 8;
+  constexpr int PER = 2 * kQGroup * SEG / 128;  // segments per thread (8 at D = 128)
+  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int col = (threadIdx.x % SEG) * 8;
+  const int r0 = blk * 2 * kQGroup;
+  uint4 xr[PER];
 #pragma unroll
-  for (int i = 0; i < SEG; ++i) {
-    const int s = lane + 32 * i;
-    const int row = r0 + s / SEG, col = (s % SEG) * 8;
-    x[i] = row < N ? ldg16(q + b * sb + (int64_t)row * sn + h * sh + col) : make_uint4(0, 0, 0, 0);
-    float f[8];
-    unpack_bf16x8(x[i], f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+  for (int i = 0; i < PER; ++i) {
+    const int row = r0 + (threadIdx.x + 128 * i) / SEG;
+    xr[i] = row < N ? ldg16(q + b * sb + (int64_t)row * sn + h * sh + col) : make_uint4(0, 0, 0, 0);
   }
-  amax = warp_max(amax);
-  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-  if (lane == 0 && g < G32)
-    q_scale[(size_t)(b * H + h) * G32 + g] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+  float am[2] = {0.0f, 0.0f};
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    float f[8];
+    unpack_bf16x8(xr[i], f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) am[i / (PER / 2)] = fmaxf(am[i / (PER / 2)], fabsf(f[j]));
+  }
+  __shared__ float red[2][4];
+  am[0] = warp_max(am[0]);
+  am[1] = warp_max(am[1]);
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = am[0];
+    red[1][threadIdx.x >> 5] = am[1];
+  }
+  __syncthreads();
+  float inv[2];
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const float a = fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3]));
+    inv[g] = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    const int grp = 2 * blk + g;
+    if (threadIdx.x == 0 && grp < G32)
+      q_scale[(size_t)(b * H + h) * G32 + grp] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+  }
   int8_t* dst = q8 + ((size_t)(b * H + h) * Nq + r0) * D;
 #pragma unroll
-  for (int i = 0; i < SEG; ++i) {
-    const int s = lane + 32 * i;
-    const int row = s / SEG, col = (s % SEG) * 8;
+  for (int i = 0; i < PER; ++i) {
+    const int r = (threadIdx.x + 128 * i) / SEG;
+    const float iv = inv[i / (PER / 2)];
     float f[8];
-    unpack_bf16x8(x[i], f);
+    unpack_bf16x8(xr[i], f);  // pad rows were loaded as zeros: zero codes
     uint2 o;
-    o.x = i8_code(f[0], inv) | i8_code(f[1], inv) << 8 | i8_code(f[2], inv) << 16 | i8_code(f[3], inv) << 24;
-    o.y = i8_code(f[4], inv) | i8_code(f[5], inv) << 8 | i8_code(f[6], inv) << 16 | i8_code(f[7], inv) << 24;
-    *reinterpret_cast<uint2*>(dst + (size_t)row * D + col) = o;
+    o.x = i8_code(f[0], iv) | i8_code(f[1], iv) << 8 | i8_code(f[2], iv) << 16 | i8_code(f[3], iv) << 24;
+    o.y = i8_code(f[4], iv) | i8_code(f[5], iv) << 8 | i8_code(f[6], iv) << 16 | i8_code(f[7], iv) << 24;
+    *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
   }
 }
 
@@ -163,7 +228,9 @@ __global__ void __launch_bounds__(128, 8) quant_k_kernel(const uint16_t* __restr
                                                          float* __restrict__ k_scale) {
   constexpr int SEG = D / 8;
   constexpr int PER = kKTile * SEG / 128;
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // heads in the reverse of the statistics pass's order: the K rows it read
+  // last are still in L2
+  const int t = blockIdx.x, h = H - 1 - (int)blockIdx.y, b = (int)gridDim.z - 1 - (int)blockIdx.z;
   const int col = (threadIdx.x % SEG) * 8;
   uint4 xr[PER];
 #pragma unroll
@@ -225,12 +292,14 @@ template <int D>
 __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict__ v, int64_t sb,
                                                       int64_t sn, int64_t sh, int N, int H, int Nk,
                                                       const float* __restrict__ v_amax,
-                                                      uint8_t* __restrict__ v8) {
+                                                      uint8_t* __restrict__ v8, float* __restrict__ v_scale) {
   constexpr int SEG = D / 8;                   // 16-byte chunks per token row
   constexpr int LOADS = kVTokens * SEG / 256;  // chunks staged per thread
   constexpr int RUNS = D * (kVTokens / 16) / 256;  // 16-token runs converted per thread
   __shared__ __align__(16) uint4 tile[kVTokens * SEG];
-  const int h = blockIdx.y, b = blockIdx.z;
+  // heads in the reverse of the statistics pass's order (its last rows are
+  // still in L2)
+  const int h = H - 1 - (int)blockIdx.y, b = (int)gridDim.z - 1 - (int)blockIdx.z;
   const int n0 = blockIdx.x * kVTokens;
   const uint16_t* vp = v + b * sb + h * sh;
   uint4 x[LOADS];
@@ -259,6 +328,8 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict
     const int ch = cb * 8 + cl;
     const float a = am[ch];
     const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
+    if (n0 == 0 && t0 == 0)  // the channel's scale, once per head
+      v_scale[(size_t)(b * H + h) * D + ch] = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
     const uint16_t* col = ts + (cb ^ q) * 8 + cl;
     uint32_t w[4];
 #pragma unroll
@@ -279,43 +350,42 @@ int check_launch() { return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_E
 
 template <int D>
 int prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int8_t* q8,
-               float* q_scale, int8_t* k8, float* k_scale, float* k_mean, double* k_part,
-               cudaStream_t s) {
+               float* q_scale, int8_t* k8, float* k_scale, float* k_mean, double* k_part, cudaStream_t s) {
   const int Nq = ceil_div(N, kQTile) * kQTile, T64 = ceil_div(N, kKTile), Nk = T64 * kKTile;
   const int G32 = ceil_div(N, kQGroup);
   const uint16_t* qp = static_cast<const uint16_t*>(q.data);
   const uint16_t* kp = static_cast<const uint16_t*>(k.data);
   constexpr int CPB = 128 / (D / 8);
-  chunk_stats_kernel<D, true, false><<<dim3(ceil_div(T64, CPB), H, B), 128, 0, s>>>(
-      kp, k.stride_b, k.stride_n, k.stride_h, nullptr, 0, 0, 0, N, H, T64, k_part, nullptr);
-  reduce_stats_kernel<true, false><<<B * H, D, 0, s>>>(N, D, T64, k_part, k_mean, nullptr, nullptr,
-                                                       nullptr);
-  quant_q_kernel<D><<<dim3(Nq / kQTile, H, B), 128, 0, s>>>(qp, q.stride_b, q.stride_n, q.stride_h,
-                                                            N, H, Nq, G32, q8, q_scale);
+  k_sums_kernel<D><<<dim3(ceil_div(T64, CPB), H, B), 128, 0, s>>>(kp, k.stride_b, k.stride_n, k.stride_h, N, H,
+                                                                  T64, k_part);
+  launch_k_mean<D>(B * H, N, T64, k_part, k_mean, s);
+  // K right after its statistics (part of K is still in L2), then Q
   quant_k_kernel<D><<<dim3(T64, H, B), 128, 0, s>>>(kp, k.stride_b, k.stride_n, k.stride_h, N, H,
                                                     Nk, T64, k_mean, k8, k_scale);
+  quant_q_kernel<D><<<dim3(Nq / (2 * kQGroup), H, B), 128, 0, s>>>(qp, q.stride_b, q.stride_n, q.stride_h,
+                                                                   N, H, Nq, G32, q8, q_scale);
   return check_launch();
 }
 
 template <int D>
-int prepass_v(const sage_view_bf16& v, int B, int N, int H, uint8_t* v8, float* v_scale,
-              float* v_part, float* v_amax, cudaStream_t s) {
+int prepass_v(const sage_view_bf16& v, int B, int N, int H, uint8_t* v8, float* v_scale, float* v_amax,
+              cudaStream_t s) {
   const int T64 = ceil_div(N, kKTile), Nk = T64 * kKTile;
   const uint16_t* vp = static_cast<const uint16_t*>(v.data);
   constexpr int CPB = 128 / (D / 8);
-  chunk_stats_kernel<D, false, true><<<dim3(ceil_div(T64, CPB), H, B), 128, 0, s>>>(
-      nullptr, 0, 0, 0, vp, v.stride_b, v.stride_n, v.stride_h, N, H, T64, nullptr, v_part);
-  reduce_stats_kernel<false, true><<<B * H, D, 0, s>>>(N, D, T64, nullptr, nullptr, v_part, v_scale,
-                                                       v_amax);
+  if (cudaMemsetAsync(v_amax, 0, sizeof(float) * (size_t)B * H * D, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  v_amax_kernel<D><<<dim3(ceil_div(T64, CPB), H, B), 128, 0, s>>>(vp, v.stride_b, v.stride_n, v.stride_h, N, H,
+                                                                  T64, v_amax);
   quant_v_kernel<D><<<dim3(ceil_div(Nk, kVTokens), H, B), 256, 0, s>>>(vp, v.stride_b, v.stride_n,
-                                                                       v.stride_h, N, H, Nk, v_amax, v8);
+                                                                       v.stride_h, N, H, Nk, v_amax, v8, v_scale);
   return check_launch();
 }
 
 }  // namespace
 
 void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s) {
-  reduce_stats_kernel<true, false><<<BH, D, 0, s>>>(N, D, T64, k_part, k_mean, nullptr, nullptr, nullptr);
+  if (D == 128) launch_k_mean<128>(BH, N, T64, k_part, k_mean, s);
+  else if (D == 64) launch_k_mean<64>(BH, N, T64, k_part, k_mean, s);
 }
 
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
@@ -327,9 +397,9 @@ int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, i
 }
 
 int launch_prepass_v(const sage_view_bf16& v, int B, int N, int H, int D, uint8_t* v8,
-                     float* v_scale, float* v_part, float* v_amax, cudaStream_t s) {
-  if (D == 128) return prepass_v<128>(v, B, N, H, v8, v_scale, v_part, v_amax, s);
-  if (D == 64) return prepass_v<64>(v, B, N, H, v8, v_scale, v_part, v_amax, s);
+                     float* v_scale, float* v_amax, cudaStream_t s) {
+  if (D == 128) return prepass_v<128>(v, B, N, H, v8, v_scale, v_amax, s);
+  if (D == 64) return prepass_v<64>(v, B, N, H, v8, v_scale, v_amax, s);
   return SAGE_ERR_UNSUPPORTED;
 }
 

@@ -95,7 +95,7 @@ Layout plan(int op, const Dims& d) {
   const bool all3 = op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QKV;
   if (all3 || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
   if (all3 || op == SAGE_OP_QUANT_V) {
-    L.v_part = take(bh * d.T64 * d.D * sizeof(float));
+    if (op == SAGE_OP_QUANT_QKV) L.v_part = take(bh * d.T64 * d.D * sizeof(float));  // single-launch prepass
     L.v_amax = take(bh * d.D * sizeof(float));
   }
   if (op == SAGE_OP_QUANT_QKV) L.counters = take((1 + 2 * bh) * sizeof(int));
@@ -236,9 +236,7 @@ int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_b
   // the separate prepass kernels: faster than the single-launch one (measured)
   if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
     return rc;
-  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_part),
-                             at<float>(workspace, L.v_amax), s)))
-    return rc;
+  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_amax), s))) return rc;
   return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
                                   out_stride_h, sm_scale, status),
                       s);
@@ -350,8 +348,7 @@ int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, f
   if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
-  return launch_prepass_v(v, B, N, H, D, v_fp8, v_scale, at<float>(workspace, L.v_part),
-                          at<float>(workspace, L.v_amax), s);
+  return launch_prepass_v(v, B, N, H, D, v_fp8, v_scale, at<float>(workspace, L.v_amax), s);
 }
 
 int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, int N, int H, int D,

@@ -139,11 +139,12 @@ void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, f
 bool prepass_fused_fits(int B, int N, int H, int D);
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s);
+// k_part: B*H*T64*D doubles of scratch; v_amax: B*H*D floats (scratch, cleared by the launch)
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,
                       double* k_part, cudaStream_t s);
 int launch_prepass_v(const sage_view_bf16& v, int B, int N, int H, int D, uint8_t* v8,
-                     float* v_scale, float* v_part, float* v_amax, cudaStream_t s);
+                     float* v_scale, float* v_amax, cudaStream_t s);
 int launch_attn_mma(const AttnParams& p, cudaStream_t s);
 int launch_debug_qk_mma(const AttnParams& p, int b, int h, int q_tile, int k_tile, int32_t* s_out,
                         cudaStream_t s);

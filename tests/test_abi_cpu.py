@@ -43,7 +43,8 @@ def test_workspace_sizes(lib):
     n = sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FWD, 1, 37810, 56, 128)
     bh, Nq, Nk, T = 56, 37888, 37824, 591
     quant = bh * (Nq * 128 + Nk * 128 + 128 * Nk)
-    assert quant + bh * T * 128 * 12 < n < quant + bh * T * 128 * 12 + (2 << 20)
+    # the quantised tensors, FP64 K partials per 64-token chunk and channel, and small vectors
+    assert quant + bh * T * 128 * 8 < n < quant + bh * T * 128 * 8 + (2 << 20)
     assert sage.sage_workspace_bytes(sage.SAGE_OP_ATTN_FROM_QUANT, 1, 37810, 56, 128) < 4096
     assert sage.sage_workspace_bytes(sage.SAGE_OP_QUANT_QK, 2, 1000, 8, 64) >= 2 * 8 * 16 * 64 * 8
     lay = sage.sage_fwd_workspace_layout(1, 1000, 8, 128)

@@ -470,7 +470,7 @@ def main():
                     "call": f"sage_attn_fwd_host: chunks of 2, 2, then {hpc}, then 2 heads on "
                             f"{'one compute stream' if args.e2e_one_stream else 'two compute streams'}, "
                             "copies overlapped with compute"},
-            "gpu_launches": args.steps * 6,  # five prepass kernels and the mainloop
+            "gpu_launches": args.steps * 7,  # six prepass kernels and the mainloop
             "clocks": clocks,
         }
         if not args.no_cpu_baseline:

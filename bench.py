@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--config", default="long_fused",
                     choices=["small", "ragged", "outlier", "long_fused", "d64_batch"])
     ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
+    ap.add_argument("--prepass", default="separate", choices=["separate", "qkv"],
+                    help="separate: sage_quant_qk + sage_quant_v (the kernels sage_attn_fwd runs); "
+                         "qkv: sage_quant_qkv (the single cooperative kernel where it applies)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=4)
     ap.add_argument("--e2e-one-stream", action="store_true", help="all chunks on one compute stream")
@@ -352,16 +355,26 @@ def main():
     dts = [torch.int8, torch.float32, torch.int8, torch.float32, torch.float32, torch.uint8,
            torch.float32]
     qt = {n: torch.empty(s, dtype=dt, device=dev) for (n, s), dt in zip(shp.items(), dts)}
-    ws_qk = sage.workspace(sage.SAGE_OP_QUANT_QK, B, N, H, D, dev)
-    ws_v = sage.workspace(sage.SAGE_OP_QUANT_V, B, N, H, D, dev)
+    if args.prepass == "qkv":
+        ws_pre = [sage.workspace(sage.SAGE_OP_QUANT_QKV, B, N, H, D, dev)]
+        pre_kernels = sage.sage_quant_qkv_kernels(B, N, H, D)
+    else:
+        ws_pre = [sage.workspace(sage.SAGE_OP_QUANT_QK, B, N, H, D, dev),
+                  sage.workspace(sage.SAGE_OP_QUANT_V, B, N, H, D, dev)]
+        pre_kernels = 6
     ws_m = sage.workspace(sage.SAGE_OP_ATTN_FROM_QUANT, B, N, H, D, dev)
     stream = torch.cuda.current_stream()
 
     def step(ev_s=None, ev_a=None, ev_b=None):
         if ev_s is not None:
             ev_s.record(stream)
-        sage.sage_quant_qk(q, k, qt["q_i8"], qt["q_scale"], qt["k_i8"], qt["k_scale"], qt["k_mean"], ws_qk)
-        sage.sage_quant_v(v, qt["v_fp8"], qt["v_scale"], ws_v)
+        if args.prepass == "qkv":
+            sage.sage_quant_qkv(q, k, v, qt["q_i8"], qt["q_scale"], qt["k_i8"], qt["k_scale"], qt["k_mean"],
+                                qt["v_fp8"], qt["v_scale"], ws_pre[0])
+        else:
+            sage.sage_quant_qk(q, k, qt["q_i8"], qt["q_scale"], qt["k_i8"], qt["k_scale"], qt["k_mean"],
+                               ws_pre[0])
+            sage.sage_quant_v(v, qt["v_fp8"], qt["v_scale"], ws_pre[1])
         if ev_a is not None:
             ev_a.record(stream)
         sage.sage_attn_from_quant(qt["q_i8"], qt["q_scale"], qt["k_i8"], qt["k_scale"], qt["v_fp8"],
@@ -376,7 +389,7 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    for w in (ws_qk, ws_v, ws_m):
+    for w in (*ws_pre, ws_m):
         st = sage.sage_read_device_status(w)
         if st != sage.SAGE_OK:
             raise RuntimeError(f"device status after warm-up: {sage.sage_strerror(st)}")
@@ -396,7 +409,7 @@ def main():
             t1.record(stream)
             torch.cuda.synchronize()
             barrier()
-        for w in (ws_qk, ws_v, ws_m):
+        for w in (*ws_pre, ws_m):
             st = sage.sage_read_device_status(w)
             if st != sage.SAGE_OK:
                 raise RuntimeError(f"device status after the timed steps: {sage.sage_strerror(st)}")
@@ -453,6 +466,8 @@ def main():
             "data": "synthetic (seeded normal BF16 stand-in for the pages' video-DiT activations)",
             "config": {"workload": f"{cfg.name}: {cfg.about}", "B": B, "N": N, "H": H, "D": D,
                        "mainloop": ml_name, "parallelism": f"{world} independent replicas",
+                       "prepass": ("single cooperative kernel" if pre_kernels == 1 else
+                                   f"{pre_kernels} separate kernels"),
                        "l2": "inputs 1.6 GB > 126 MB L2 (no flush needed)"
                        if cfg.name == "long_fused" else "see workload"},
             "mainloop_ms": ml_avg, "mainloop_ms_min": min(ml_ms), "prepass_ms": ms_step - ml_avg,
@@ -470,7 +485,7 @@ def main():
                     "call": f"sage_attn_fwd_host: chunks of 2, 2, then {hpc}, then 2 heads on "
                             f"{'one compute stream' if args.e2e_one_stream else 'two compute streams'}, "
                             "copies overlapped with compute"},
-            "gpu_launches": args.steps * 7,  # six prepass kernels and the mainloop
+            "gpu_launches": args.steps * (pre_kernels + 1),  # the prepass kernels and the mainloop
             "clocks": clocks,
         }
         if not args.no_cpu_baseline:

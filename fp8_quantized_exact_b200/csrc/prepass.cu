@@ -9,29 +9,13 @@
 // Contract" (per-warp INT8 Q in 32-row groups, per-block INT8 K with 64-row
 // blocks, FP8 V with a per-channel scale).  The exact rounding steps follow
 // the readings stated in include/sage_b200.h.
-#include "sage_common.cuh"
+#include "prepass_codes.cuh"
 
 namespace sage {
 namespace {
 
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) {
   return __ldg(reinterpret_cast<const uint4*>(p));
-}
-
-// INT8 code of one product, round half to even, clamped to +-127.
-__device__ __forceinline__ uint32_t i8_code(float x, float inv) {
-  int r = __float2int_rn(__fmul_rn(x, inv));
-  r = max(-127, min(127, r));
-  return static_cast<uint32_t>(r) & 0xFFu;
 }
 
 // ------------------------------------------------------------------------
@@ -177,30 +161,56 @@ __global__ void __launch_bounds__(128, 6) quant_q_kernel(const uint16_t* __restr
     const int row = r0 + (threadIdx.x + 128 * i) / SEG;
     xr[i] = row < N ? ldg16(q + b * sb + (int64_t)row * sn + h * sh + col) : make_uint4(0, 0, 0, 0);
   }
-  float am[2] = {0.0f, 0.0f};
+  // amax as BF16 magnitude bits (NaN and inf above every finite value)
+  uint32_t mb[2] = {0u, 0u};
 #pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    float f[8];
-    unpack_bf16x8(xr[i], f);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) am[i / (PER / 2)] = fmaxf(am[i / (PER / 2)], fabsf(f[j]));
-  }
+  for (int i = 0; i < PER; ++i) mb[i / (PER / 2)] = amax_bits8(xr[i], mb[i / (PER / 2)]);
+  __shared__ uint32_t redb[2][4];
   __shared__ float red[2][4];
-  am[0] = warp_max(am[0]);
-  am[1] = warp_max(am[1]);
+#pragma unroll
+  for (int g = 0; g < 2; ++g) mb[g] = __reduce_max_sync(0xffffffffu, halves_max(mb[g]));
   if ((threadIdx.x & 31) == 0) {
-    red[0][threadIdx.x >> 5] = am[0];
-    red[1][threadIdx.x >> 5] = am[1];
+    redb[0][threadIdx.x >> 5] = mb[0];
+    redb[1][threadIdx.x >> 5] = mb[1];
   }
   __syncthreads();
-  float inv[2];
+  float a[2];
+  bool finite[2];
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    const float a = fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3]));
-    inv[g] = a > 0.0f ? __fdiv_rn(127.0f, a) : 0.0f;
+    mb[g] = max(max(redb[g][0], redb[g][1]), max(redb[g][2], redb[g][3]));
+    finite[g] = mb[g] < 0x7F80u;
+    a[g] = __uint_as_float(mb[g] << 16);
+  }
+  if (!finite[0] || !finite[1]) {
+    // NaN or inf in the block: the amax that ignores NaN (the reference form)
+    float am[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      float f[8];
+      unpack_bf16x8(xr[i], f);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) am[i / (PER / 2)] = fmaxf(am[i / (PER / 2)], fabsf(f[j]));
+    }
+    am[0] = warp_max(am[0]);
+    am[1] = warp_max(am[1]);
+    if ((threadIdx.x & 31) == 0) {
+      red[0][threadIdx.x >> 5] = am[0];
+      red[1][threadIdx.x >> 5] = am[1];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < 2; ++g) a[g] = fmaxf(fmaxf(red[g][0], red[g][1]), fmaxf(red[g][2], red[g][3]));
+  }
+  float inv[2];
+  bool fast[2];
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    inv[g] = a[g] > 0.0f ? __fdiv_rn(127.0f, a[g]) : 0.0f;
+    fast[g] = finite[g] && codes_fast(a[g], inv[g]);
     const int grp = 2 * blk + g;
     if (threadIdx.x == 0 && grp < G32)
-      q_scale[(size_t)(b * H + h) * G32 + grp] = a > 0.0f ? __fdiv_rn(a, 127.0f) : 0.0f;
+      q_scale[(size_t)(b * H + h) * G32 + grp] = a[g] > 0.0f ? __fdiv_rn(a[g], 127.0f) : 0.0f;
   }
   int8_t* dst = q8 + ((size_t)(b * H + h) * Nq + r0) * D;
 #pragma unroll
@@ -209,9 +219,7 @@ __global__ void __launch_bounds__(128, 6) quant_q_kernel(const uint16_t* __restr
     const float iv = inv[i / (PER / 2)];
     float f[8];
     unpack_bf16x8(xr[i], f);  // pad rows were loaded as zeros: zero codes
-    uint2 o;
-    o.x = i8_code(f[0], iv) | i8_code(f[1], iv) << 8 | i8_code(f[2], iv) << 16 | i8_code(f[3], iv) << 24;
-    o.y = i8_code(f[4], iv) | i8_code(f[5], iv) << 8 | i8_code(f[6], iv) << 16 | i8_code(f[7], iv) << 24;
+    const uint2 o = fast[i / (PER / 2)] ? i8_codes8_fast(f, iv) : i8_codes8_ref(f, iv);
     *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
   }
 }
@@ -249,15 +257,38 @@ __global__ void __launch_bounds__(128, 8) quant_k_kernel(const uint16_t* __restr
       float f[8];
       unpack_bf16x8(xr[i], f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fsub_rn(f[j], km[j])));
+      for (int j = 0; j < 8; ++j) amax = fmax_nan(amax, fabsf(__fsub_rn(f[j], km[j])));
     }
   }
+  // the bits of non-negative floats order as integers, NaN above inf
+  __shared__ uint32_t redb[4];
   __shared__ float red[4];
-  amax = warp_max(amax);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  uint32_t ab = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+  if ((threadIdx.x & 31) == 0) redb[threadIdx.x >> 5] = ab;
   __syncthreads();
-  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  ab = max(max(redb[0], redb[1]), max(redb[2], redb[3]));
+  const bool finite = ab < 0x7F800000u;
+  amax = __uint_as_float(ab);
+  if (!finite) {
+    // NaN or inf in the block: the amax that ignores NaN (the reference form)
+    amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int row = t * kKTile + (threadIdx.x + 128 * i) / SEG;
+      if (row < N) {
+        float f[8];
+        unpack_bf16x8(xr[i], f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fsub_rn(f[j], km[j])));
+      }
+    }
+    amax = warp_max(amax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  }
   const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  const bool fast = finite && codes_fast(amax, inv);
   if (threadIdx.x == 0)
     k_scale[(size_t)(b * H + h) * T64 + t] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
   int8_t* dst = k8 + ((size_t)(b * H + h) * Nk + (size_t)t * kKTile) * D;
@@ -271,8 +302,7 @@ __global__ void __launch_bounds__(128, 8) quant_k_kernel(const uint16_t* __restr
       float x[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) x[j] = __fsub_rn(f[j], km[j]);
-      o.x = i8_code(x[0], inv) | i8_code(x[1], inv) << 8 | i8_code(x[2], inv) << 16 | i8_code(x[3], inv) << 24;
-      o.y = i8_code(x[4], inv) | i8_code(x[5], inv) << 8 | i8_code(x[6], inv) << 16 | i8_code(x[7], inv) << 24;
+      o = fast ? i8_codes8_fast(x, inv) : i8_codes8_ref(x, inv);
     }
     *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
   }

@@ -1,62 +1,75 @@
 // Single-launch prepass: K channel mean, Q/K INT8 and V E4M3 quantisation in
-// one persistent kernel, with each head's K and V read from HBM once and
-// re-read from L2 for the quantisation.
+// one cooperative kernel in which every byte of Q, K and V is read from HBM
+// once.
 //
 // Operation: the same steps and rounding as the separate prepass kernels
 // ("Sage2 Blackwell Mainloop", sections "Decision" and "Existing
-// Contract"); the fusion of the producers follows the pages' P1/P2 producer
-// fusions ("Sage2 Blackwell Mainloop", section "Completed P1 And P2").  The
-// bytes and scales are identical to the separate kernels: the FP64 K sums
-// run in token order inside each 64-token chunk and the chunk partials are
-// added in chunk order by one thread per channel.
+// Contract"), fused into one producer as the pages' P1/P2 producer fusions
+// do ("Sage2 Blackwell Mainloop", section "Completed P1 And P2").  Bytes and
+// scales equal those of the separate kernels.
 //
-// Work is handed out by a global ticket in head-major order, in slots; slot
-// s holds, for head s, nS statistics items (CPI chunks of 64 tokens each:
-// FP64 K sums and V amax partials; the CTA that completes the head's last
-// chunk reduces the partials to k_mean, v_amax and v_scale and raises the
-// head flag) and nQ Q items (16 groups of 32 rows each), and for head
-// s - kLookahead its nS K/V items (CPI chunks: wait for the head flag, then
-// K smoothing and INT8 K, E4M3 V stored transposed).  The lookahead gives
-// the statistics of a head time to finish before its K/V items are taken,
-// while the K and V of the heads in flight (about 20 MB each) stay in L2.
-// A K/V item only ever waits for statistics items with smaller tickets,
-// which running CTAs have already claimed and finish without waiting, so
-// the waits always end; they are bounded all the same (the status word
-// records SAGE_ERR_TIMEOUT and the item is skipped).
+// Layout of the work.  One CTA per SM (grid G <= SM count, a cooperative
+// launch, so all CTAs are resident together).  CTA i owns a fixed run of
+// 64-token chunks, [i*T64/G, (i+1)*T64/G), in every head; its slice of one
+// head is at most 64 KB.  Heads (units u = b*H + h) are taken g at a time
+// ("groups") in two passes, K with Q, then V.  At step s a CTA:
+//   1. starts the copy of the slices of step s+1 into shared memory
+//      (cp.async, three 64 KB slots);
+//   2. computes the statistics of the slices of step s (K: FP64 sums, V:
+//      absolute maxima) and publishes them with atomics, then counts itself
+//      in for each unit of the group;
+//   3. in the K pass, quantises the Q rows of its chunks (plain loads issued
+//      at the start of the step);
+//   4. waits (bounded) until all G CTAs have counted in for the group of
+//      step s-1, and quantises that group's K or V slices, which are still
+//      in shared memory.
+// So K and V are read once, and the statistics of one group overlap the
+// quantisation of the previous one.
+//
+// The K mean.  The definition is the FP64 sum of the FP64 chunk partials
+// in chunk order, each partial a token-order FP64 sum, divided by N in FP64
+// and rounded once to FP32.  When every addition in that chain is exact,
+// any order and grouping of the additions gives the same bits.  A BF16 value
+// of biased exponent e is a multiple of 2^(max(e,1)-134), and its magnitude
+// is below 2^(e-126).  Take emax and emin, the largest and smallest such e
+// (emin over the nonzero values, with e taken as at least 1).  Every partial
+// sum of a channel is then a multiple of 2^(emin-134) and below
+// N * 2^(emax-126) in magnitude.  It is exactly representable in FP64 when
+// ceil(log2 N) + emax <= emin + 45.  Each CTA therefore adds its local
+// (exact) sum into an FP64 accumulator with an atomic add, and publishes
+// emax and 255 - emin with atomic maxima.  A channel that meets the bound
+// takes its mean from the accumulator.  For a channel that does not, the
+// CTAs add the chunk partials (written to k_part) in chunk order, one warp
+// per channel.  Every CTA computes the same means; CTA 0 stores them.
+//
+// Waits.  A CTA only waits for counts that every CTA reaches without
+// waiting on anything itself: the statistics of step s come before its wait
+// at step s.  Each wait is bounded (the status word records
+// SAGE_ERR_TIMEOUT, a global abort flag stops the others, and every CTA
+// leaves after draining its own copies).
 #include <algorithm>
 
-#include "sage_common.cuh"
+#include "prepass_codes.cuh"
 
 namespace sage {
 namespace {
 
-constexpr int kThreadsP = 256;
-constexpr int kQPerItem = 16;  // 32-row Q groups per Q item (two per warp)
-constexpr int kLookahead = 2;  // heads between a head's statistics and its K/V items
+constexpr int kRThreads = 512;
+constexpr int kCtasPerSm = 2;
+constexpr int kSlotBytes = 32 * 1024;
+constexpr int kSlots = 3;
+constexpr int kMaxSliceChunkD = kSlotBytes / (kKTile * 2);  // max chunks x D of one slice (256)
 
-__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-__device__ __forceinline__ uint4 ld16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-
-__device__ __forceinline__ uint32_t code_i8(float x, float inv) {
-  int r = __float2int_rn(__fmul_rn(x, inv));
-  r = max(-127, min(127, r));
-  return static_cast<uint32_t>(r) & 0xFFu;
-}
-
-struct FusedArgs {
+struct ResArgs {
   const uint16_t *q, *k, *v;
   int64_t qsb, qsn, qsh, ksb, ksn, ksh, vsb, vsn, vsh;
-  int B, N, H, Nq, Nk, T64, G32, Gq;  // Gq: 32-row groups of the padded Q (Nq / 32)
-  int nS, nQ, per_head;              // items per head: nS stats, nQ Q, nS K/V
-  int BH;
+  int N, H, U, Nq, Nk, T64, TQ, G32;
+  int G;      // CTAs
+  int g;      // units per group
+  int S;      // groups per pass
+  int cpc;    // most K/V chunks of one CTA
+  int cpcq;   // most Q chunks of one CTA
+  int log2t;  // ceil(log2 T64)
   int8_t* q8;
   float* q_scale;
   int8_t* k8;
@@ -64,396 +77,722 @@ struct FusedArgs {
   float* k_mean;
   uint8_t* v8;
   float* v_scale;
-  float* v_amax;
-  double* k_part;
-  float* v_part;
-  int* ticket;     // [1]
-  int* head_done;  // [B*H] chunks whose statistics are written
-  int* head_flag;  // [B*H] 1 once k_mean / v_amax of the head are written
+  double* k_part;  // [U][T64][D] FP64 chunk partials (read only for channels off the bound)
+  double* k_sum;   // [U][D] zeroed
+  int* k_hi;       // [U][D] zeroed: kExpBias + max over chunks of floor(log2 |partial|)
+  int* k_lov;      // [U][D] zeroed: kExpBias - min over chunks of the lowest set bit (0: all partials 0)
+  int* v_amax;     // [U][D] zeroed: FP32 bits of the channel amax
+  int* arrive;     // [2][U] zeroed: CTAs counted in (K, V)
+  int* abort_flag; // [1] zeroed
   DeviceStatus* status;
   long long wait_limit;
+  int stall_unit;  // test hook: CTA 0 does not count in for the K of this unit (-1: none)
 };
 
-// ------------------------------------------------------------ statistics
-// Threads 0..127: K sums, threads 128..255: V amax; D/8 threads per chunk,
-// each owning 8 consecutive channels.
+__device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+
+
+// Shared-memory image of a slice: token rows of D BF16 values; the 16-byte
+// piece k of row r is stored at position k ^ ((r >> 4) & 3), so that reads
+// down a channel (16 tokens per lane, four 16-token runs per warp) and reads
+// along a row both fall in distinct banks.
 template <int D>
-__device__ void stats_item(const FusedArgs& a, int bh, int c0, int c1) {
-  constexpr int TPC = D / 8;
-  const int half = threadIdx.x >> 7, t = threadIdx.x & 127;
-  const int chunk = c0 + t / TPC, col = (t % TPC) * 8;
-  const int b = bh / a.H, h = bh % a.H;
-  if (chunk < c1) {
-    const int n0 = chunk * kKTile, n1 = min(n0 + kKTile, a.N);
-    const size_t o = ((size_t)bh * a.T64 + chunk) * D + col;
-    if (half == 0) {
-      double ks[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ks[i] = 0.0;
-      const uint16_t* kp = a.k + b * a.ksb + h * a.ksh + col;
-#pragma unroll 16
-      for (int n = n0; n < n1; ++n) {
-        float f[8];
-        unpack8(ld16(kp + n * a.ksn), f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) ks[i] = __dadd_rn(ks[i], (double)f[i]);
-      }
-      double2* dst = reinterpret_cast<double2*>(a.k_part + o);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) dst[i] = make_double2(ks[2 * i], ks[2 * i + 1]);
-    } else {
-      float vm[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) vm[i] = 0.0f;
-      const uint16_t* vp = a.v + b * a.vsb + h * a.vsh + col;
-#pragma unroll 16
-      for (int n = n0; n < n1; ++n) {
-        float f[8];
-        unpack8(ld16(vp + n * a.vsn), f);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) vm[i] = fmaxf(vm[i], fabsf(f[i]));
-      }
-      float4* dst = reinterpret_cast<float4*>(a.v_part + o);
-      dst[0] = make_float4(vm[0], vm[1], vm[2], vm[3]);
-      dst[1] = make_float4(vm[4], vm[5], vm[6], vm[7]);
+__device__ __forceinline__ uint32_t slice_off(int r, int piece) {
+  return (uint32_t)(r * D * 2 + ((piece ^ ((r >> 4) & 3)) << 4));
+}
+
+struct Range {
+  int lo, n;  // first chunk and chunk count of this CTA
+};
+__device__ __forceinline__ Range cta_range(int total, int G) {
+  const int i = blockIdx.x;
+  const int lo = (int)((long long)i * total / G), hi = (int)((long long)(i + 1) * total / G);
+  return {lo, hi - lo};
+}
+
+// Copies of the K (kind 0) or V (kind 1) slices of group grp into a slot,
+// issued by the Q warps only: the statistics warps, whose thread 0 releases
+// the CTA's counts, then have no copies in flight for that release to wait
+// on.
+template <int D>
+__device__ void issue_slices(const ResArgs& a, int kind, int grp, uint8_t* slot, Range r) {
+  constexpr int SEG = D / 8;
+  const uint16_t* base = kind == 0 ? a.k : a.v;
+  const int64_t sb = kind == 0 ? a.ksb : a.vsb, sn = kind == 0 ? a.ksn : a.vsn, sh = kind == 0 ? a.ksh : a.vsh;
+  if (threadIdx.x < kRThreads / 2) return;  // statistics warps
+  const int per_unit = r.n * kKTile * SEG;
+  const uint32_t s0 = smem_u32(slot);
+  for (int i = 0; i < a.g; ++i) {
+    const int u = grp * a.g + i;
+    if (u >= a.U) break;
+    const uint16_t* ub = base + (u / a.H) * sb + (u % a.H) * sh;
+    const uint32_t sd = s0 + (uint32_t)(i * a.cpc * kKTile * D * 2);
+    for (int idx = threadIdx.x - kRThreads / 2; idx < per_unit; idx += kRThreads / 2) {
+      const int row = idx / SEG, piece = idx % SEG;
+      const int n = r.lo * kKTile + row;
+      const bool valid = n < a.N;
+      cp_async_16_zfill(sd + slice_off<D>(row, piece), valid ? ub + (int64_t)n * sn + piece * 8 : base, valid);
     }
   }
-  // count the chunks; the CTA that completes the head reduces it
-  __shared__ int last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&a.head_done[bh], c1 - c0) + (c1 - c0) == a.T64;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  if (threadIdx.x < D) {
-    const int d = threadIdx.x;
-    // partials added in chunk order; loads fetched 16 ahead of the adds
-    const double* src = a.k_part + (size_t)bh * a.T64 * D + d;
-    double total = 0.0;
-    for (int c0 = 0; c0 < a.T64; c0 += 16) {
-      double x[16];
+}
+
+// Warps 0-7 ("statistics warps") and warps 8-15 ("Q warps") synchronise
+// among themselves with named barriers while the other half works.
+constexpr int kHalf = kRThreads / 2;
+constexpr int kBarStats = 1, kBarQ = 2;
+__device__ __forceinline__ void bar_half(int id) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kHalf) : "memory"); }
+
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));  // a NaN operand yields the other
+  return d;
+}
+
+// Bounded wait (thread 0) until all CTAs have counted in for every unit of a
+// group; the statistics warps then pass a named barrier.  Returns false (in
+// every statistics thread) when the wait ran out or another CTA gave up.
+__device__ bool wait_group(const ResArgs& a, int kind, int grp, int* s_flag) {
+  if (threadIdx.x == 0) {
+    int good = 1;
+    for (int i = 0; i < a.g && good; ++i) {
+      const int u = grp * a.g + i;
+      if (u >= a.U) break;
+      const int* cnt = a.arrive + kind * a.U + u;
+      const long long t0 = clock64();
+      for (unsigned it = 0;; ++it) {
+        int c;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(c) : "l"(cnt) : "memory");
+        if (c >= a.G) break;
+        if (*reinterpret_cast<volatile int*>(a.abort_flag)) {
+          good = 0;
+          break;
+        }
+        if (clock64() - t0 > a.wait_limit) {
+          good = 0;
+          if (atomicCAS(&a.status->code, 0, (int)SAGE_ERR_TIMEOUT) == 0) {
+            a.status->where = 40 + kind;
+            a.status->block = (int)blockIdx.x;
+          }
+          atomicExch(a.abort_flag, 1);
+          break;
+        }
+        __nanosleep(it < 8 ? 32 : 256);
+      }
+    }
+    *s_flag = good;
+  }
+  bar_half(kBarStats);
+  return *s_flag != 0;
+}
+
+// Count this CTA in for each unit of the group.  Called by the statistics
+// warps after a named barrier that follows all their writes and atomics:
+// thread 0's release is cumulative over what the barrier ordered before it.
+__device__ void count_in(const ResArgs& a, int kind, int grp) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < a.g; ++i) {
+      const int u = grp * a.g + i;
+      if (u >= a.U) break;
+      if (kind == 0 && u == a.stall_unit && blockIdx.x == 0) continue;
+      int* cnt = a.arrive + kind * a.U + u;
+      asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(cnt) : "memory");
+    }
+  }
+}
+
+// ------------------------------------------------------------ statistics
+// Statistics thread t < 256 takes channels d, d+1 (d even) of one chunk of
+// one unit: the two FP64 token-order sums (K) or absolute maxima (V).
+// Rows come 16 at a time, whose pieces share one swizzle.
+//
+// K also reports, per channel, floor(log2 |p|) and the exponent of the
+// lowest set bit of each nonzero chunk partial p (atomic maxima of kExpBias
+// + hi and kExpBias - lo), which the K mean's exactness test needs.
+constexpr int kExpBias = 1100;
+
+__device__ __forceinline__ void partial_bits(double p, int& hi, int& lo) {
+  // p is a nonzero sum of BF16 values: a normal FP64 number
+  const unsigned long long bits = (unsigned long long)__double_as_longlong(p);
+  const int e = (int)((bits >> 52) & 0x7FFu);
+  const unsigned long long sig = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+  hi = e - 1023;
+  lo = e - 1075 + __ffsll((long long)sig) - 1;
+}
+
+template <int D>
+__device__ __noinline__ void k_stats(const ResArgs& a, int grp, const uint8_t* slot, Range r, double* sp) {
+  const int t = threadIdx.x;
+  const int item = t / (D / 2), d = 2 * (t % (D / 2));
+  const int i = item / a.cpc, cc = item % a.cpc;
+  const int u = grp * a.g + i;
+  double p0 = 0.0, p1 = 0.0;
+  if (i < a.g && u < a.U && cc < r.n) {
+    const uint8_t* s = slot + i * a.cpc * kKTile * D * 2 + ((d & 7) << 1);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = c0 + j < a.T64 ? __ldcg(src + (size_t)(c0 + j) * D) : 0.0;
+    for (int r0 = cc * kKTile; r0 < cc * kKTile + kKTile; r0 += 16) {
+      const uint8_t* rp = s + slice_off<D>(r0, d >> 3);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {  // token order; pad rows hold zeros
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(rp + j * D * 2);
+        p0 = __dadd_rn(p0, (double)__uint_as_float(w << 16));
+        p1 = __dadd_rn(p1, (double)__uint_as_float(w & 0xFFFF0000u));
+      }
+    }
+    *reinterpret_cast<double2*>(a.k_part + ((size_t)u * a.T64 + r.lo + cc) * D + d) = make_double2(p0, p1);
+  }
+  if (item < a.g * a.cpc) {
+    sp[item * D + d] = p0;
+    sp[item * D + d + 1] = p1;
+  }
+  bar_half(kBarStats);
+  if (t < a.g * D / 2) {
+    const int i2 = t / (D / 2), d2 = 2 * (t % (D / 2)), u2 = grp * a.g + i2;
+    if (u2 < a.U) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        double sum = 0.0;
+        int hi = 0, lov = 0;
+        for (int c = 0; c < r.n; ++c) {  // the CTA's chunks in order
+          const double p = sp[(i2 * a.cpc + c) * D + d2 + h];
+          sum = __dadd_rn(sum, p);
+          if (p != 0.0) {
+            int ph, pl;
+            partial_bits(p, ph, pl);
+            hi = max(hi, kExpBias + ph);
+            lov = max(lov, kExpBias - pl);
+          }
+        }
+        const size_t at = (size_t)u2 * D + d2 + h;
+        atomicAdd(a.k_sum + at, sum);
+        if (lov) {
+          atomicMax(a.k_hi + at, hi);
+          atomicMax(a.k_lov + at, lov);
+        }
+      }
+    }
+  }
+  bar_half(kBarStats);
+}
+
+template <int D>
+__device__ __noinline__ void v_stats(const ResArgs& a, int grp, const uint8_t* slot, Range r, float* sf) {
+  const int t = threadIdx.x;
+  const int item = t / (D / 2), d = 2 * (t % (D / 2));
+  const int i = item / a.cpc, cc = item % a.cpc;
+  const int u = grp * a.g + i;
+  uint32_t m = 0u;
+  if (i < a.g && u < a.U && cc < r.n) {
+    const uint8_t* s = slot + i * a.cpc * kKTile * D * 2 + ((d & 7) << 1);
+#pragma unroll
+    for (int r0 = cc * kKTile; r0 < cc * kKTile + kKTile; r0 += 16) {
+      const uint8_t* rp = s + slice_off<D>(r0, d >> 3);
 #pragma unroll
       for (int j = 0; j < 16; ++j)
-        if (c0 + j < a.T64) total = __dadd_rn(total, x[j]);
+        m = max_bf16x2(m, *reinterpret_cast<const uint32_t*>(rp + j * D * 2) & 0x7FFF7FFFu);
     }
-    a.k_mean[(size_t)bh * D + d] = __double2float_rn(__ddiv_rn(total, (double)a.N));
-  } else if (threadIdx.x >= 128 && threadIdx.x < 128 + D) {
-    const int d = threadIdx.x - 128;
-    const float* src = a.v_part + (size_t)bh * a.T64 * D + d;
-    float am = 0.0f;
-    for (int c0 = 0; c0 < a.T64; c0 += 16) {
-      float x[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = c0 + j < a.T64 ? __ldcg(src + (size_t)(c0 + j) * D) : 0.0f;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) am = fmaxf(am, x[j]);
-    }
-    a.v_amax[(size_t)bh * D + d] = am;
-    a.v_scale[(size_t)bh * D + d] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) atomicExch(&a.head_flag[bh], 1);
+  if (item < a.g * a.cpc) {
+    sf[item * D + d] = __uint_as_float(m << 16);
+    sf[item * D + d + 1] = __uint_as_float(m & 0xFFFF0000u);
+  }
+  bar_half(kBarStats);
+  if (t < a.g * D / 2) {
+    const int i2 = t / (D / 2), d2 = 2 * (t % (D / 2)), u2 = grp * a.g + i2;
+    if (u2 < a.U) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float mxv = 0.0f;
+        for (int c = 0; c < r.n; ++c) mxv = fmaxf(mxv, sf[(i2 * a.cpc + c) * D + d2 + h]);
+        // the amax of non-negative floats is exact in any order, and their
+        // bit patterns order as integers
+        if (mxv > 0.0f) atomicMax(a.v_amax + (size_t)u2 * D + d2 + h, __float_as_int(mxv));
+      }
+    }
+  }
+  bar_half(kBarStats);
 }
 
 // ---------------------------------------------------------------------- Q
-// One warp per 32-row group, two groups per warp; pad rows and pad groups
-// of the padded Q get zero bytes.
+// The Q warps (256 threads): D threads per 64-row chunk, 8 pieces of 16
+// bytes each (pieces tt + D * j: rows tt/(D/8) + 8j, so j < 4 lie in the
+// first 32-row group and j >= 4 in the second).  The loads are issued at the
+// start of the step and used after the K slice has arrived.
+constexpr int kQPieces = 8;
+
 template <int D>
-__device__ void q_item(const FusedArgs& a, int bh, int g0) {
-  constexpr int SEG = D / 8;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = bh / a.H, h = bh % a.H;
-#pragma unroll 1
-  for (int k = 0; k < 2; ++k) {
-    const int g = g0 + 2 * warp + k;
-    if (g >= a.Gq) break;
-    const int r0 = g * kQGroup;
-    uint4 x[SEG];
-    float amax = 0.0f;
+__device__ void q_load(const ResArgs& a, int grp, Range rq, uint4 (&x)[kQPieces]) {
+  constexpr int SEG = D / 8, TPI = D;
+  const int qt = threadIdx.x - kHalf;
+  const int item = qt / TPI, tt = qt % TPI, col = (tt % SEG) * 8;
+  const int i = item / a.cpcq, cc = item % a.cpcq;
+  const int u = grp * a.g + i;
+  const bool live = i < a.g && u < a.U && cc < rq.n;
+  const int b = live ? u / a.H : 0, h = live ? u % a.H : 0;
 #pragma unroll
-    for (int i = 0; i < SEG; ++i) {
-      const int s = lane + 32 * i;
-      const int row = r0 + s / SEG, col = (s % SEG) * 8;
-      x[i] = row < a.N ? ld16(a.q + b * a.qsb + (int64_t)row * a.qsn + h * a.qsh + col) : make_uint4(0, 0, 0, 0);
+  for (int j = 0; j < kQPieces; ++j) {
+    const int row = (rq.lo + cc) * kKTile + tt / SEG + 8 * j;
+    x[j] = live && row < a.N ? ldg16(a.q + b * a.qsb + (int64_t)row * a.qsn + h * a.qsh + col)
+                             : make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int D>
+__device__ void q_quant(const ResArgs& a, int grp, Range rq, const uint4 (&x)[kQPieces], uint32_t* redq,
+                        int* s_any) {
+  constexpr int SEG = D / 8, TPI = D, WPI = TPI / 32, HALF = kQPieces / 2;
+  const int qt = threadIdx.x - kHalf, qw = qt >> 5, lane = qt & 31;
+  const int item = qt / TPI, tt = qt % TPI, col = (tt % SEG) * 8;
+  const int i = item / a.cpcq, cc = item % a.cpcq;
+  const int u = grp * a.g + i;
+  const bool live = i < a.g && u < a.U && cc < rq.n;
+  // amax as BF16 magnitude bits (NaN and inf above every finite value)
+  uint32_t mb[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < kQPieces; ++j) mb[j / HALF] = amax_bits8(x[j], mb[j / HALF]);
+  mb[0] = __reduce_max_sync(0xffffffffu, halves_max(mb[0]));
+  mb[1] = __reduce_max_sync(0xffffffffu, halves_max(mb[1]));
+  if (qt == 0) *s_any = 0;
+  if (lane == 0) {
+    redq[2 * qw] = mb[0];
+    redq[2 * qw + 1] = mb[1];
+  }
+  bar_half(kBarQ);
+  float am[2];
+  bool finite[2];
+#pragma unroll
+  for (int gg = 0; gg < 2; ++gg) {
+    uint32_t m = redq[2 * (item * WPI) + gg];
+#pragma unroll
+    for (int w = 1; w < WPI; ++w) m = max(m, redq[2 * (item * WPI + w) + gg]);
+    finite[gg] = m < 0x7F80u;
+    am[gg] = __uint_as_float(m << 16);
+    if (!finite[gg]) *s_any = 1;
+  }
+  bar_half(kBarQ);
+  if (*s_any) {
+    // NaN or inf among the rows: the amax that ignores NaN (the reference form)
+    float af[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int j = 0; j < kQPieces; ++j) {
       float f[8];
-      unpack8(x[i], f);
+      unpack_bf16x8(x[j], f);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[j]));
+      for (int e = 0; e < 8; ++e) af[j / HALF] = fmaxf(af[j / HALF], fabsf(f[e]));
     }
-    amax = warp_max(amax);
-    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-    if (lane == 0 && g < a.G32) a.q_scale[(size_t)bh * a.G32 + g] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-    int8_t* dst = a.q8 + ((size_t)bh * a.Nq + r0) * D;
+    af[0] = warp_max(af[0]);
+    af[1] = warp_max(af[1]);
+    float* redf = reinterpret_cast<float*>(redq) + 16;
+    if (lane == 0) {
+      redf[2 * qw] = af[0];
+      redf[2 * qw + 1] = af[1];
+    }
+    bar_half(kBarQ);
 #pragma unroll
-    for (int i = 0; i < SEG; ++i) {
-      const int s = lane + 32 * i;
-      const int row = s / SEG, col = (s % SEG) * 8;
+    for (int gg = 0; gg < 2; ++gg) {
+      float m = redf[2 * (item * WPI) + gg];
+#pragma unroll
+      for (int w = 1; w < WPI; ++w) m = fmaxf(m, redf[2 * (item * WPI + w) + gg]);
+      am[gg] = m;
+    }
+  }
+  float inv[2];
+  bool fast[2];
+#pragma unroll
+  for (int gg = 0; gg < 2; ++gg) {
+    inv[gg] = am[gg] > 0.0f ? __fdiv_rn(127.0f, am[gg]) : 0.0f;
+    fast[gg] = finite[gg] && codes_fast(am[gg], inv[gg]);
+    const int grp32 = 2 * (rq.lo + cc) + gg;
+    if (live && tt == 0 && grp32 < a.G32)
+      a.q_scale[(size_t)u * a.G32 + grp32] = am[gg] > 0.0f ? __fdiv_rn(am[gg], 127.0f) : 0.0f;
+  }
+  if (live) {
+    int8_t* dst = a.q8 + ((size_t)u * a.Nq + (size_t)(rq.lo + cc) * kKTile) * D + col;
+#pragma unroll
+    for (int j = 0; j < kQPieces; ++j) {
+      const int rr = tt / SEG + 8 * j;
       float f[8];
-      unpack8(x[i], f);
-      uint2 o;
-      o.x = code_i8(f[0], inv) | code_i8(f[1], inv) << 8 | code_i8(f[2], inv) << 16 | code_i8(f[3], inv) << 24;
-      o.y = code_i8(f[4], inv) | code_i8(f[5], inv) << 8 | code_i8(f[6], inv) << 16 | code_i8(f[7], inv) << 24;
-      *reinterpret_cast<uint2*>(dst + (size_t)row * D + col) = o;
+      unpack_bf16x8(x[j], f);  // pad rows were loaded as zeros: zero codes
+      *reinterpret_cast<uint2*>(dst + (size_t)rr * D) =
+          fast[j / HALF] ? i8_codes8_fast(f, inv[j / HALF]) : i8_codes8_ref(f, inv[j / HALF]);
     }
   }
 }
 
-// -------------------------------------------------------------------- K/V
-// Wait (bounded) for the head's statistics; returns false on timeout.
-__device__ bool wait_head(const FusedArgs& a, int bh) {
-  __shared__ int ok;
-  if (threadIdx.x == 0) {
-    const long long t0 = clock64();
-    int f = 0;
-    for (unsigned i = 0;; ++i) {
-      asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(f) : "l"(a.head_flag + bh) : "memory");
-      if (f) break;
-      if (clock64() - t0 > a.wait_limit) break;
-      __nanosleep(i < 16 ? 64 : 256);
-    }
-    ok = f;
-    if (!f && atomicCAS(&a.status->code, 0, (int)SAGE_ERR_TIMEOUT) == 0) {
-      a.status->where = 30;
-      a.status->block = (int)blockIdx.x;
+// ------------------------------------------------------------------ K mean
+// Statistics warps: the mean of every channel of the group's units into
+// mean_s[i * D + d] (all CTAs compute the same values; CTA 0 stores them).
+template <int D>
+__device__ __noinline__ void k_means(const ResArgs& a, int grp, float* mean_s, int* list, int* s_cnt) {
+  const int t = threadIdx.x;
+  if (t == 0) *s_cnt = 0;
+  bar_half(kBarStats);
+  for (int c = t; c < a.g * D; c += kHalf) {
+    const int u = grp * a.g + c / D;
+    if (u >= a.U) break;
+    const size_t at = (size_t)u * D + c % D;
+    const int hi = __ldcg(a.k_hi + at) - kExpBias, lov = __ldcg(a.k_lov + at);
+    // every partial is a multiple of 2^lo and below 2^(hi+1) in magnitude, so
+    // every sum of partials is a multiple of 2^lo below 2^(log2t + hi + 1):
+    // exact in FP64 when log2t + hi - lo <= 52, and then the accumulator
+    // holds the chunk-order sum (all partials zero: +0)
+    if (lov == 0 || a.log2t + hi - (kExpBias - lov) <= 52) {
+      mean_s[c] = lov == 0 ? 0.0f : __double2float_rn(__ddiv_rn(__ldcg(a.k_sum + at), (double)a.N));
+    } else {
+      list[atomicAdd(s_cnt, 1)] = c;
     }
   }
-  __syncthreads();
-  return ok != 0;
+  bar_half(kBarStats);
+  const int nlist = *s_cnt;
+  if (nlist > 0) {
+    // channels off the bound: the chunk partials added in chunk order, one
+    // warp per channel (lanes load 32 chunks at a time; every lane adds the
+    // same values in the same order, so all hold the same total)
+    const int warp = t >> 5, lane = t & 31;
+    for (int e = warp; e < nlist; e += kHalf / 32) {
+      const int c = list[e];
+      const int u = grp * a.g + c / D, d = c % D;
+      const double* src = a.k_part + (size_t)u * a.T64 * D + d;
+      double total = 0.0;
+      double nxt = lane < a.T64 ? __ldcg(src + (size_t)lane * D) : 0.0;
+      for (int c0 = 0; c0 < a.T64; c0 += 32) {
+        const double cur = nxt;
+        if (c0 + 32 + lane < a.T64) nxt = __ldcg(src + (size_t)(c0 + 32 + lane) * D);
+        const int n = min(32, a.T64 - c0);
+        for (int j = 0; j < n; ++j) total = __dadd_rn(total, __shfl_sync(0xffffffffu, cur, j));
+      }
+      if (lane == 0) mean_s[c] = __double2float_rn(__ddiv_rn(total, (double)a.N));
+    }
+    bar_half(kBarStats);
+  }
+  if (blockIdx.x == 0)
+    for (int c = t; c < a.g * D; c += kHalf) {
+      const int u = grp * a.g + c / D;
+      if (u < a.U) a.k_mean[(size_t)u * D + c % D] = mean_s[c];
+    }
 }
 
-// K: 128 threads per 64-row chunk, two chunks at a time; x' = fl32(x - km).
-// The raw BF16 chunks stay in registers between the amax and code passes.
+// Statistics warps: 448 / amax of every channel of the group's units into
+// vinv_s (CTA 0 also stores the scales amax / 448).
 template <int D>
-__device__ void k_quant(const FusedArgs& a, int bh, int c0, int c1) {
-  constexpr int SEG = D / 8;
-  constexpr int PER = kKTile * SEG / 128;
-  const int half = threadIdx.x >> 7, t = threadIdx.x & 127;
-  const int b = bh / a.H, h = bh % a.H;
-  const int col = (t % SEG) * 8;
-  float km[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) km[j] = __ldcg(a.k_mean + (size_t)bh * D + col + j);
-  __shared__ float red[8];
-#pragma unroll 1
-  for (int cb = c0; cb < c1; cb += 2) {
-    const int chunk = cb + half;
-    const bool live = chunk < c1;
+__device__ void v_scales(const ResArgs& a, int grp, float* vinv_s) {
+  for (int c = threadIdx.x; c < a.g * D; c += kHalf) {
+    const int u = grp * a.g + c / D;
+    if (u >= a.U) break;
+    const float am = __int_as_float(__ldcg(a.v_amax + (size_t)u * D + c % D));
+    vinv_s[c] = am > 0.0f ? __fdiv_rn(448.0f, am) : 0.0f;
+    if (blockIdx.x == 0) a.v_scale[(size_t)u * D + c % D] = am > 0.0f ? __fdiv_rn(am, 448.0f) : 0.0f;
+  }
+}
+
+// K: 2D threads per 64-row chunk (all chunks of a step at once) from the
+// resident slice; x' = fl32(x - km).
+template <int D>
+__device__ void k_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r, const float* kmean_s, float* red,
+                        int* s_any) {
+  constexpr int SEG = D / 8, TPI = 2 * D, WPI = TPI / 32, IPP = kRThreads / TPI;
+  constexpr int PER = kKTile * SEG / TPI;  // 4
+  const int tt = threadIdx.x % TPI, piece = tt % SEG, col = piece * 8;
+  uint32_t* redb = reinterpret_cast<uint32_t*>(red);
+  const int items = a.g * a.cpc;
+  for (int it0 = 0; it0 < items; it0 += IPP) {
+    const int item = it0 + threadIdx.x / TPI;
+    const int i = item / a.cpc, cc = item % a.cpc;
+    const int u = grp * a.g + i;
+    const bool live = item < items && u < a.U && cc < r.n;
     uint4 xr[PER];
+    float km[8];
+    float amax = 0.0f;  // NaN-propagating
+    if (live) {
+      const uint8_t* s = slot + i * a.cpc * kKTile * D * 2;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int row = chunk * kKTile + (t + 128 * i) / SEG;
-      xr[i] = live && row < a.N ? ld16(a.k + b * a.ksb + (int64_t)row * a.ksn + h * a.ksh + col)
-                                : make_uint4(0, 0, 0, 0);
-    }
-    float amax = 0.0f;
+      for (int j = 0; j < 8; ++j) km[j] = kmean_s[i * D + col + j];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int row = chunk * kKTile + (t + 128 * i) / SEG;
-      if (live && row < a.N) {
-        float f[8];
-        unpack8(xr[i], f);
+      for (int p = 0; p < PER; ++p) {
+        const int rr = (tt + TPI * p) / SEG;
+        xr[p] = *reinterpret_cast<const uint4*>(s + slice_off<D>(cc * kKTile + rr, piece));
+        if ((r.lo + cc) * kKTile + rr < a.N) {
+          float f[8];
+          unpack_bf16x8(xr[p], f);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(__fsub_rn(f[j], km[j])));
+          for (int j = 0; j < 8; ++j) amax = fmax_nan(amax, fabsf(__fsub_rn(f[j], km[j])));
+        }
       }
     }
-    amax = warp_max(amax);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+    // the bits of non-negative floats order as integers, NaN above inf
+    const uint32_t ab = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
+    if (threadIdx.x == 0) *s_any = 0;
+    if ((threadIdx.x & 31) == 0) redb[threadIdx.x >> 5] = ab;
     __syncthreads();
-    amax = fmaxf(fmaxf(red[4 * half], red[4 * half + 1]), fmaxf(red[4 * half + 2], red[4 * half + 3]));
+    const uint32_t* rb = redb + (threadIdx.x / TPI) * WPI;
+    uint32_t m = rb[0];
+#pragma unroll
+    for (int w = 1; w < WPI; ++w) m = max(m, rb[w]);
+    const bool finite = m < 0x7F800000u;
+    amax = __uint_as_float(m);
+    if (!finite) *s_any = 1;
     __syncthreads();
+    if (*s_any) {
+      // NaN or inf among the rows: the amax that ignores NaN (the reference form)
+      float af = 0.0f;
+      if (live)
+#pragma unroll
+        for (int p = 0; p < PER; ++p) {
+          const int rr = (tt + TPI * p) / SEG;
+          if ((r.lo + cc) * kKTile + rr < a.N) {
+            float f[8];
+            unpack_bf16x8(xr[p], f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) af = fmaxf(af, fabsf(__fsub_rn(f[j], km[j])));
+          }
+        }
+      af = warp_max(af);
+      if ((threadIdx.x & 31) == 0) red[16 + (threadIdx.x >> 5)] = af;
+      __syncthreads();
+      const float* rw = red + 16 + (threadIdx.x / TPI) * WPI;
+      amax = rw[0];
+#pragma unroll
+      for (int w = 1; w < WPI; ++w) amax = fmaxf(amax, rw[w]);
+    }
+    __syncthreads();  // red is reused by the next items
     if (live) {
       const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-      if (t == 0) a.k_scale[(size_t)bh * a.T64 + chunk] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-      int8_t* dst = a.k8 + ((size_t)bh * a.Nk + (size_t)chunk * kKTile) * D;
+      const bool fast = finite && codes_fast(amax, inv);
+      if (tt == 0) a.k_scale[(size_t)u * a.T64 + r.lo + cc] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+      int8_t* dst = a.k8 + ((size_t)u * a.Nk + (size_t)(r.lo + cc) * kKTile) * D;
 #pragma unroll
-      for (int i = 0; i < PER; ++i) {
-        const int r = (t + 128 * i) / SEG;
+      for (int p = 0; p < PER; ++p) {
+        const int rr = (tt + TPI * p) / SEG;
         uint2 o = make_uint2(0u, 0u);  // pad rows get zero codes
-        if (chunk * kKTile + r < a.N) {
+        if ((r.lo + cc) * kKTile + rr < a.N) {
           float f[8], x[8];
-          unpack8(xr[i], f);
+          unpack_bf16x8(xr[p], f);
 #pragma unroll
           for (int j = 0; j < 8; ++j) x[j] = __fsub_rn(f[j], km[j]);
-          o.x = code_i8(x[0], inv) | code_i8(x[1], inv) << 8 | code_i8(x[2], inv) << 16 | code_i8(x[3], inv) << 24;
-          o.y = code_i8(x[4], inv) | code_i8(x[5], inv) << 8 | code_i8(x[6], inv) << 16 | code_i8(x[7], inv) << 24;
+          o = fast ? i8_codes8_fast(x, inv) : i8_codes8_ref(x, inv);
         }
-        *reinterpret_cast<uint2*>(dst + (size_t)r * D + col) = o;
+        *reinterpret_cast<uint2*>(dst + (size_t)rr * D + col) = o;
       }
     }
   }
 }
 
-// V: 128 tokens at a time staged in shared memory with 16-byte loads (the
-// chunk index of a row XORed with bits 4-5 of its token, so that the column
-// reads hit distinct banks); each thread then converts 16 consecutive tokens
-// of one channel to E4M3 (token t in byte t of the channel's row) and writes
-// them as one 16-byte vector.
-constexpr int kVBlock = 2 * kKTile;
-
+// V: runs of 16 tokens of one channel from the resident slice converted to
+// E4M3 (token t in byte t of the channel's row) and stored as one 16-byte
+// vector; a warp covers four runs of eight channels (64 contiguous bytes
+// per channel).
 template <int D>
-__device__ void v_quant(const FusedArgs& a, int bh, int c0, int c1) {
+__device__ void v_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r, const float* vinv_s) {
   constexpr int SEG = D / 8;
-  constexpr int LOADS = kVBlock * SEG / kThreadsP;
-  constexpr int RUNS = D * (kVBlock / 16) / kThreadsP;
-  __shared__ __align__(16) uint4 tile[kVBlock * SEG];
-  const int b = bh / a.H, h = bh % a.H;
-  const uint16_t* vp = a.v + b * a.vsb + h * a.vsh;
-  const float* am = a.v_amax + (size_t)bh * D;
-  const uint16_t* ts = reinterpret_cast<const uint16_t*>(tile);
-  const int tok1 = min(c1 * kKTile, a.Nk);  // end of this item's tokens (padded length)
-#pragma unroll 1
-  for (int n0 = c0 * kKTile; n0 < tok1; n0 += kVBlock) {
-    __syncthreads();  // the previous block's column reads are done
-    // staged in two rounds of loads, to stay within the registers
+  const int runs = a.g * a.cpc * 4 * D;
+  for (int idx = threadIdx.x; idx < runs; idx += kRThreads) {
+    const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
+    const int cb = rest % SEG, item = rest / SEG;
+    const int i = item / a.cpc, cc = item % a.cpc;
+    const int u = grp * a.g + i;
+    if (u >= a.U || cc >= r.n) continue;
+    const int ch = cb * 8 + cl;
+    const float inv = vinv_s[i * D + ch];
+    const uint8_t* s = slot + i * a.cpc * kKTile * D * 2;
+    const int t0 = cc * kKTile + 16 * q;  // (t >> 4) & 3 == q for the run's tokens
+    const uint16_t* colp = reinterpret_cast<const uint16_t*>(s + (((cb ^ q) << 4) + (cl << 1)));
+    uint32_t w[4];
 #pragma unroll
-    for (int i0 = 0; i0 < LOADS; i0 += LOADS / 2) {
-      uint4 x[LOADS / 2];
-#pragma unroll
-      for (int i = 0; i < LOADS / 2; ++i) {
-        const int idx = threadIdx.x + kThreadsP * (i0 + i);
-        const int r = idx / SEG, k = idx % SEG;
-        x[i] = n0 + r < a.N ? ld16(vp + (int64_t)(n0 + r) * a.vsn + k * 8) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < LOADS / 2; ++i) {
-        const int idx = threadIdx.x + kThreadsP * (i0 + i);
-        const int r = idx / SEG, k = idx % SEG;
-        tile[r * SEG + (k ^ ((r >> 4) & 3))] = x[i];
-      }
+    for (int j = 0; j < 4; ++j) {
+      const int tk = t0 + 4 * j;
+      const uint32_t lo = e4m3x2(__fmul_rn(bf16_bits_to_f32(colp[tk * D]), inv),
+                                 __fmul_rn(bf16_bits_to_f32(colp[(tk + 1) * D]), inv));
+      const uint32_t hi = e4m3x2(__fmul_rn(bf16_bits_to_f32(colp[(tk + 2) * D]), inv),
+                                 __fmul_rn(bf16_bits_to_f32(colp[(tk + 3) * D]), inv));
+      w[j] = inv > 0.0f ? (lo | (hi << 16)) : 0u;
     }
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < RUNS; ++i) {
-      const int idx = threadIdx.x + kThreadsP * i;
-      const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
-      const int cb = rest % SEG, hf = rest / SEG;
-      const int t0 = hf * kKTile + 16 * q;
-      if (n0 + hf * kKTile >= tok1) continue;
-      const int ch = cb * 8 + cl;
-      const float amx = __ldcg(am + ch);
-      const float inv = amx > 0.0f ? __fdiv_rn(448.0f, amx) : 0.0f;
-      const uint16_t* col = ts + (cb ^ q) * 8 + cl;
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = t0 + 4 * j;
-        const uint32_t lo = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[t * D]), inv),
-                                   __fmul_rn(bf16_bits_to_f32(col[(t + 1) * D]), inv));
-        const uint32_t hi = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[(t + 2) * D]), inv),
-                                   __fmul_rn(bf16_bits_to_f32(col[(t + 3) * D]), inv));
-        w[j] = amx > 0.0f ? (lo | (hi << 16)) : 0u;
-      }
-      uint8_t* dst = a.v8 + ((size_t)bh * D + ch) * a.Nk + n0 + t0;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
+    uint8_t* dst = a.v8 + ((size_t)u * D + ch) * a.Nk + (size_t)(r.lo + cc) * kKTile + 16 * q;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
+// Dynamic shared memory: the slots, then the scratch.
+constexpr size_t kScratchOff = (size_t)kSlots * kSlotBytes;
+constexpr size_t kSmemBytes = kScratchOff + kMaxSliceChunkD * sizeof(double)  // sp (FP64 partials / FP32 maxima)
+                              + kMaxSliceChunkD * sizeof(float)                // mean_s (K means / V 448/amax)
+                              + kMaxSliceChunkD * sizeof(int)                  // list
+                              + 64 * sizeof(float);                            // red (K: 32), redq (Q: 32)
+
+// Step st (0 <= st <= 2S): statistics of group st (K for st < S, V after)
+// and, in the K pass, the Q rows of group st; then the quantisation of
+// group st - 1 from its resident slices.
 template <int D>
-__global__ void __launch_bounds__(kThreadsP, 2) prepass_fused_kernel(const FusedArgs a) {
-  constexpr int CPI = 128 / (D / 8);  // chunks per statistics or K/V item
-  __shared__ int item_s;
-  // a slot of the ticket sequence: statistics and Q items of head s, then
-  // the K/V items of head s - kLookahead (either part may be absent)
-  const int total = (a.BH + kLookahead) * a.per_head;
-  for (;;) {
-    __syncthreads();
-    if (threadIdx.x == 0) item_s = atomicAdd(a.ticket, 1);
-    __syncthreads();
-    const int item = item_s;
-    if (item >= total) break;
-    const int slot = item / a.per_head, r = item % a.per_head;
-    if (r < a.nS + a.nQ) {
-      const int bh = slot;
-      if (bh >= a.BH) continue;
-      if (r < a.nS) stats_item<D>(a, bh, r * CPI, min(a.T64, (r + 1) * CPI));
-      else q_item<D>(a, bh, (r - a.nS) * kQPerItem);
-    } else {
-      const int bh = slot - kLookahead;
-      if (bh < 0) continue;
-      const int u = r - a.nS - a.nQ;
-      if (!wait_head(a, bh)) continue;
-      const int c0 = u * CPI, c1 = min(a.T64, (u + 1) * CPI);
-      k_quant<D>(a, bh, c0, c1);
-      v_quant<D>(a, bh, c0, c1);
+__global__ void __launch_bounds__(kRThreads, kCtasPerSm) prepass_resident_kernel(const __grid_constant__ ResArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  double* sp = reinterpret_cast<double*>(smem + kScratchOff);
+  float* mean_s = reinterpret_cast<float*>(sp + kMaxSliceChunkD);
+  int* list = reinterpret_cast<int*>(mean_s + kMaxSliceChunkD);
+  float* red = reinterpret_cast<float*>(list + kMaxSliceChunkD);
+  uint32_t* redq = reinterpret_cast<uint32_t*>(red + 32);
+  __shared__ int s_flag, s_cnt, s_anyq, s_anyk;
+
+  const Range rk = cta_range(a.T64, a.G);
+  const Range rq = cta_range(a.TQ, a.G);
+  const int total = 2 * a.S;
+  const bool stats_warp = threadIdx.x < kHalf;
+  auto slot = [&](int st) { return smem + (size_t)(st % kSlots) * kSlotBytes; };
+
+  if (threadIdx.x == 0) s_flag = 1;
+  issue_slices<D>(a, 0, 0, slot(0), rk);
+  cp_async_commit();
+  for (int st = 0; st <= total; ++st) {
+    if (st + 1 < total) issue_slices<D>(a, st + 1 < a.S ? 0 : 1, (st + 1) % a.S, slot(st + 1), rk);
+    cp_async_commit();
+    const bool kstep = st < a.S;
+    uint4 qx[kQPieces];
+    if (!stats_warp && kstep) q_load<D>(a, st, rq, qx);
+    cp_async_wait<1>();
+    __syncthreads();  // the slices of step st are in (every thread's copies)
+    if (stats_warp) {
+      if (st < total) {
+        if (kstep) k_stats<D>(a, st, slot(st), rk, sp);
+        else v_stats<D>(a, st - a.S, slot(st), rk, reinterpret_cast<float*>(sp));
+        count_in(a, kstep ? 0 : 1, st % a.S);
+      }
+      if (st >= 1) {
+        const int pv = st - 1, kind = pv < a.S ? 0 : 1, grp = pv % a.S;
+        if (wait_group(a, kind, grp, &s_flag)) {
+          if (kind == 0) k_means<D>(a, grp, mean_s, list, &s_cnt);
+          else v_scales<D>(a, grp, mean_s);
+        }
+      }
+    } else if (kstep) {
+      q_quant<D>(a, st, rq, qx, redq, &s_anyq);
     }
+    __syncthreads();
+    if (!s_flag) {
+      cp_async_wait<0>();  // no copy may land after the CTA has left
+      return;
+    }
+    if (st >= 1) {
+      const int pv = st - 1;
+      if (pv < a.S) k_quant<D>(a, pv, slot(pv), rk, mean_s, red, &s_anyk);
+      else v_quant<D>(a, pv - a.S, slot(pv), rk, mean_s);
+    }
+    __syncthreads();  // slot (st - 1) % 3 is refilled at the next step
   }
 }
 
-// SM count of the current device (asked on every call: the runtime answers
-// from its own cache, and devices of one process may differ)
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      n <= 0)
-    n = 148;
-  return n;
+// SM count and cooperative-launch support of the current device (asked on
+// every call: the runtime answers from its own cache, and devices of one
+// process may differ).
+bool device_info(int* sms, int* coop) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) return false;
+  return *sms > 0;
 }
 
-// Work items of one call: the kernel's ticket counter and its item count are
-// int, and each CTA draws one ticket past the end before it leaves.
-constexpr long long kMaxItems = 1LL << 30;
+struct Plan {
+  int G, g, S, cpc, cpcq;
+};
 
-template <int D>
-long long fused_items(int B, int N, int H) {
-  constexpr int CPI = 128 / (D / 8);
-  const long long T64 = ceil_div(N, kKTile), Gq = ceil_div(N, kQTile) * kQTile / kQGroup;
-  const long long per_head = 2 * ((T64 + CPI - 1) / CPI) + (Gq + kQPerItem - 1) / kQPerItem;
-  return ((long long)B * H + kLookahead) * per_head;
+// Resident CTAs per SM of the kernel for D (0 on failure).
+int ctas_per_sm(int D) {
+  const void* fn = D == 128 ? reinterpret_cast<const void*>(prepass_resident_kernel<128>)
+                            : reinterpret_cast<const void*>(prepass_resident_kernel<64>);
+  int nb = 0;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, kRThreads, kSmemBytes) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return std::min(nb, kCtasPerSm);
+}
+
+// The shape's partition for `slots` resident CTAs; false when one CTA's
+// slice would not fit a slot (more than kMaxSliceChunkD chunks x channels).
+bool make_plan(int B, int N, int H, int D, int slots, Plan* p) {
+  const long long T64 = ceil_div(N, kKTile), TQ = (long long)ceil_div(N, kQTile) * (kQTile / kKTile);
+  const long long U = (long long)B * H;
+  const int G = (int)std::min<long long>(slots, T64);
+  if (G <= 0) return false;
+  const long long cpc = (T64 + G - 1) / G, cpcq = (TQ + G - 1) / G;
+  const long long span = std::max(cpc, cpcq) * D;
+  if (span > kMaxSliceChunkD) return false;
+  p->G = G;
+  p->cpc = (int)cpc;
+  p->cpcq = (int)cpcq;
+  p->g = (int)std::min<long long>(U, kMaxSliceChunkD / span);
+  p->S = (int)((U + p->g - 1) / p->g);
+  return true;
 }
 
 template <int D>
-int fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N, int H,
-          const FusedOut& o, cudaStream_t s) {
-  constexpr int CPI = 128 / (D / 8);
-  FusedArgs a;
+int resident(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N, int H,
+             const FusedOut& o, const Plan& pl, cudaStream_t s) {
+  ResArgs a;
   a.q = static_cast<const uint16_t*>(q.data);
   a.k = static_cast<const uint16_t*>(k.data);
   a.v = static_cast<const uint16_t*>(v.data);
   a.qsb = q.stride_b; a.qsn = q.stride_n; a.qsh = q.stride_h;
   a.ksb = k.stride_b; a.ksn = k.stride_n; a.ksh = k.stride_h;
   a.vsb = v.stride_b; a.vsn = v.stride_n; a.vsh = v.stride_h;
-  a.B = B; a.N = N; a.H = H;
+  a.N = N; a.H = H; a.U = B * H;
   a.Nq = ceil_div(N, kQTile) * kQTile;
   a.T64 = ceil_div(N, kKTile);
   a.Nk = a.T64 * kKTile;
+  a.TQ = a.Nq / kKTile;
   a.G32 = ceil_div(N, kQGroup);
-  a.Gq = a.Nq / kQGroup;
-  a.nS = ceil_div(a.T64, CPI);
-  a.nQ = ceil_div(a.Gq, kQPerItem);
-  a.per_head = 2 * a.nS + a.nQ;
-  a.BH = B * H;
+  a.G = pl.G; a.g = pl.g; a.S = pl.S; a.cpc = pl.cpc; a.cpcq = pl.cpcq;
+  int l2 = 0;
+  while ((1 << l2) < a.T64) ++l2;
+  a.log2t = l2;
   a.q8 = o.q8; a.q_scale = o.q_scale; a.k8 = o.k8; a.k_scale = o.k_scale; a.k_mean = o.k_mean;
-  a.v8 = o.v8; a.v_scale = o.v_scale; a.v_amax = o.v_amax; a.k_part = o.k_part; a.v_part = o.v_part;
-  a.ticket = o.counters;
-  a.head_done = o.counters + 1;
-  a.head_flag = o.counters + 1 + B * H;
+  a.v8 = o.v8; a.v_scale = o.v_scale;
+  a.k_part = o.k_part;
+  const size_t UD = (size_t)a.U * D;
+  char* sync = reinterpret_cast<char*>(o.sync);
+  a.k_sum = reinterpret_cast<double*>(sync);
+  a.k_hi = reinterpret_cast<int*>(sync + UD * 8);
+  a.k_lov = a.k_hi + UD;
+  a.v_amax = a.k_lov + UD;
+  a.arrive = a.v_amax + UD;
+  a.abort_flag = a.arrive + 2 * (size_t)a.U;
   a.status = o.status;
   a.wait_limit = o.wait_limit;
-  if (cudaMemsetAsync(o.counters, 0, sizeof(int) * (1 + 2 * (size_t)B * H), s) != cudaSuccess) return SAGE_ERR_CUDA;
-  const long long items = fused_items<D>(B, N, H);
-  if (items > kMaxItems) return SAGE_ERR_UNSUPPORTED;
-  const int grid = (int)std::min<long long>(items, 2LL * sm_count());
-  prepass_fused_kernel<D><<<grid, kThreadsP, 0, s>>>(a);
-  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+  a.stall_unit = o.stall_unit;
+  if (cudaMemsetAsync(o.sync, 0, prepass_sync_bytes(B, H, D), s) != cudaSuccess) return SAGE_ERR_CUDA;
+  const void* fn = reinterpret_cast<const void*>(prepass_resident_kernel<D>);
+  void* args[] = {&a};
+  if (cudaLaunchCooperativeKernel(fn, dim3(pl.G), dim3(kRThreads), args, kSmemBytes, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  return SAGE_OK;
 }
 
 }  // namespace
 
+size_t prepass_sync_bytes(int B, int H, int D) {
+  const size_t U = (size_t)B * H;
+  return U * D * (sizeof(double) + 3 * sizeof(int)) + (2 * U + 4) * sizeof(int);
+}
+
+// Resident CTA slots of the current device for D, or 0 when the kernel
+// cannot run there (no cooperative launch, or no room for a CTA).
+int resident_slots(int D) {
+  int sms = 0, coop = 0;
+  if ((D != 64 && D != 128) || !device_info(&sms, &coop) || !coop) return 0;
+  return sms * ctas_per_sm(D);
+}
+
 bool prepass_fused_fits(int B, int N, int H, int D) {
-  if (D != 64 && D != 128) return false;
-  return (D == 128 ? fused_items<128>(B, N, H) : fused_items<64>(B, N, H)) <= kMaxItems;
+  const int slots = resident_slots(D);
+  Plan p;
+  return slots > 0 && make_plan(B, N, H, D, slots, &p);
 }
 
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s) {
-  if (D == 128) return fused<128>(q, k, v, B, N, H, o, s);
-  if (D == 64) return fused<64>(q, k, v, B, N, H, o, s);
-  return SAGE_ERR_UNSUPPORTED;
+  const int slots = resident_slots(D);
+  Plan p;
+  if (slots <= 0 || !make_plan(B, N, H, D, slots, &p)) return SAGE_ERR_UNSUPPORTED;
+  if (D == 128) return resident<128>(q, k, v, B, N, H, o, p, s);
+  return resident<64>(q, k, v, B, N, H, o, p, s);
 }
 
 }  // namespace sage

@@ -70,7 +70,7 @@ int check_out(const void* out, int64_t sb, int64_t sn, int64_t sh) {
 struct Layout {
   size_t status = 0;
   size_t q8 = 0, q_scale = 0, k8 = 0, k_scale = 0, k_mean = 0, v8 = 0, v_scale = 0;
-  size_t k_part = 0, v_part = 0, v_amax = 0, counters = 0;
+  size_t k_part = 0, v_amax = 0, sync = 0;
   size_t total = 0;
 };
 
@@ -94,11 +94,8 @@ Layout plan(int op, const Dims& d) {
   }
   const bool all3 = op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QKV;
   if (all3 || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
-  if (all3 || op == SAGE_OP_QUANT_V) {
-    if (op == SAGE_OP_QUANT_QKV) L.v_part = take(bh * d.T64 * d.D * sizeof(float));  // single-launch prepass
-    L.v_amax = take(bh * d.D * sizeof(float));
-  }
-  if (op == SAGE_OP_QUANT_QKV) L.counters = take((1 + 2 * bh) * sizeof(int));
+  if (all3 || op == SAGE_OP_QUANT_V) L.v_amax = take(bh * d.D * sizeof(float));
+  if (op == SAGE_OP_QUANT_QKV) L.sync = take(prepass_sync_bytes(d.B, d.H, d.D));  // single-launch prepass
   L.total = off;
   return L;
 }
@@ -116,16 +113,30 @@ T* at(void* ws, size_t off) {
 }
 
 FusedOut fused_out(void* ws, const Layout& L, int8_t* q8, float* qs, int8_t* k8, float* ks, float* km,
-                   uint8_t* v8, float* vs) {
+                   uint8_t* v8, float* vs, void* status) {
   FusedOut o;
   o.q8 = q8; o.q_scale = qs; o.k8 = k8; o.k_scale = ks; o.k_mean = km; o.v8 = v8; o.v_scale = vs;
-  o.v_amax = at<float>(ws, L.v_amax);
   o.k_part = at<double>(ws, L.k_part);
-  o.v_part = at<float>(ws, L.v_part);
-  o.counters = at<int>(ws, L.counters);
-  o.status = static_cast<DeviceStatus*>(ws);
+  o.sync = at<void>(ws, L.sync);
+  o.status = static_cast<DeviceStatus*>(status);
   o.wait_limit = g_wait_limit.load();
+  o.stall_unit = g_stall_tile.load();
   return o;
+}
+
+// The three prepasses on checked arguments into the given outputs: the
+// single-launch kernel where it applies (and `single` allows it), else the
+// separate kernels.  Both give the same bytes.
+int prepass_all(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N, int H,
+                int D, int8_t* q8, float* qs, int8_t* k8, float* ks, float* km, uint8_t* v8, float* vs,
+                void* ws, const Layout& L, void* status, bool single, cudaStream_t s) {
+  int rc;
+  if (single && prepass_fused_fits(B, N, H, D)) {
+    rc = launch_prepass_fused(q, k, v, B, N, H, D, fused_out(ws, L, q8, qs, k8, ks, km, v8, vs, status), s);
+    if (rc != SAGE_ERR_UNSUPPORTED) return rc;
+  }
+  if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(ws, L.k_part), s))) return rc;
+  return launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(ws, L.v_amax), s);
 }
 
 int clear_status(void* ws, cudaStream_t s) {
@@ -222,7 +233,7 @@ bool device_memory(const void* p) {
 // callers clear).
 int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, void* out,
              int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N, int H, int D,
-             float sm_scale, void* workspace, void* status, cudaStream_t s) {
+             float sm_scale, void* workspace, void* status, bool single_prepass, cudaStream_t s) {
   int rc;
   const Dims d = make_dims(B, N, H, D);
   const Layout L = plan(SAGE_OP_ATTN_FWD, d);
@@ -233,10 +244,8 @@ int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_b
   float* km = at<float>(workspace, L.k_mean);
   uint8_t* v8 = at<uint8_t>(workspace, L.v8);
   float* vs = at<float>(workspace, L.v_scale);
-  // the separate prepass kernels: faster than the single-launch one (measured)
-  if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(workspace, L.k_part), s)))
+  if ((rc = prepass_all(q, k, v, B, N, H, D, q8, qs, k8, ks, km, v8, vs, workspace, L, status, single_prepass, s)))
     return rc;
-  if ((rc = launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(workspace, L.v_amax), s))) return rc;
   return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
                                   out_stride_h, sm_scale, status),
                       s);
@@ -357,7 +366,6 @@ int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, 
   int rc = check_dims(B, N, H, D);
   if (rc) return rc;
   if (empty(B, N, H)) return SAGE_OK;
-  if (!prepass_fused_fits(B, N, H, D)) return SAGE_ERR_UNSUPPORTED;
   if ((rc = check_view(q)) || (rc = check_view(k)) || (rc = check_view(v))) return rc;
   if (!q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean || !v_fp8 || !v_scale) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(q_scale) || !aligned16(k_scale) ||
@@ -368,8 +376,15 @@ int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, 
   if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
-  return launch_prepass_fused(q, k, v, B, N, H, D,
-                              fused_out(workspace, L, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale), s);
+  return prepass_all(q, k, v, B, N, H, D, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale, workspace, L,
+                     workspace, true, s);
+}
+
+int sage_quant_qkv_kernels(int B, int N, int H, int D) {
+  const int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return 0;
+  return prepass_fused_fits(B, N, H, D) ? 1 : 6;
 }
 
 int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
@@ -407,8 +422,10 @@ int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* ou
   if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
+  // the separate prepass kernels: faster than the single launch on B200
+  // (0.65 against 1.3 ms at B1 N37810 H56 D128)
   return fwd_body(q, k, v, out, out_stride_b, out_stride_n, out_stride_h, B, N, H, D, sm_scale, workspace,
-                  workspace, s);
+                  workspace, false, s);
 }
 
 int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_bf16 v_host,
@@ -479,8 +496,11 @@ int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_b
       cv[i].data = static_cast<const uint16_t*>(dv[i]->data) + (int64_t)h0 * dv[i]->stride_h;
     }
     void* co = static_cast<uint16_t*>(out_dev) + (int64_t)h0 * out_stride_h;
+    // the separate prepass kernels: chunks of a few heads on two streams,
+    // overlapping other chunks' mainloops (a cooperative launch would
+    // contend with those for co-residency)
     if ((rc = fwd_body(cv[0], cv[1], cv[2], co, out_stride_b, out_stride_n, out_stride_h, B, N, h1 - h0, D,
-                       sm_scale, wsc, workspace, sc)))
+                       sm_scale, wsc, workspace, false, sc)))
       return rc;
     if (!ok(cudaEventRecord(e_comp, sc)) || !ok(cudaStreamWaitEvent(s_out, e_comp, 0))) return SAGE_ERR_CUDA;
     if ((rc = copy_heads(out_host, out_dev, out_stride_b, out_stride_n, out_stride_h, B, N, D, h0, h1,

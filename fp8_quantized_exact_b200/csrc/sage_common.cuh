@@ -115,12 +115,11 @@ struct FusedOut {
   float* k_mean;
   uint8_t* v8;
   float* v_scale;
-  float* v_amax;       // [B][H][D]
   double* k_part;      // [B][H][T64][D]
-  float* v_part;       // [B][H][T64][D]
-  int* counters;       // 1 + 2*B*H ints, zeroed by the launcher
+  void* sync;          // prepass_sync_bytes(B, H, D), zeroed by the launcher
   DeviceStatus* status;
   long long wait_limit;
+  int stall_unit;      // test hook (-1: none)
 };
 // Inputs of the RMSNorm + RoPE producer (device pointers).
 struct NormRopeIn {
@@ -134,8 +133,11 @@ int launch_norm_rope_qk(const NormRopeIn& in, const sage_view_bf16& q, const sag
                         int D, int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean, double* k_part,
                         cudaStream_t s);
 void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s);
-// false when the single-launch prepass would need more work items than its
-// int ticket counter allows (B*H*N beyond about 1.8e11)
+// Bytes of the single-launch prepass's zeroed scratch (statistics
+// accumulators and arrival counters).
+size_t prepass_sync_bytes(int B, int H, int D);
+// true when the single-launch prepass applies to the shape on the current
+// device (cooperative launch, one CTA's slice of a head within 64 KB)
 bool prepass_fused_fits(int B, int N, int H, int D);
 int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                          int H, int D, const FusedOut& o, cudaStream_t s);

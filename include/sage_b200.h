@@ -34,8 +34,7 @@
  *   - Shapes: B (batch), N (tokens), H (heads), D (head dim, 64 or 128).
  *     B, N or H equal to 0 is an empty problem: SAGE_OK, nothing launched.
  *     Limits (SAGE_ERR_UNSUPPORTED beyond them): B <= 65535 and H <= 65535
- *     (grid extents), B*H <= 2^30, N <= 2^28; sage_quant_qkv also needs
- *     B*H*N below about 1.8e11 (D = 128) or 2.7e11 (D = 64).
+ *     (grid extents), B*H <= 2^30, N <= 2^28.
  *   - BF16 views carry element strides (b, n, h); d has unit stride.  The
  *     base address and every stride must be 16-byte aligned (strides a
  *     multiple of 8 elements); three views may alias one fused projection
@@ -162,21 +161,43 @@ SAGE_API int sage_norm_rope_quant_qk(sage_view_bf16 q, sage_view_bf16 k, const v
 SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t* v_fp8, float* v_scale,
                  void* workspace, size_t workspace_bytes, void* stream);
 
-/* All three prepasses in one launch: the outputs of sage_quant_qk and
- * sage_quant_v, bit for bit (same K sum order, same rounding).  Each head's
- * K and V are read from HBM once; the quantisation re-reads them from L2
- * (the pages' producer fusions, "Sage2 Blackwell Mainloop", section
- * "Completed P1 And P2").  A persistent kernel takes work in head-major
- * order; the K/V quantisation of a head waits, bounded, for the head's
- * statistics (a wait that runs out leaves SAGE_ERR_TIMEOUT in the status
- * word).  On one B200 it is slower than the two separate calls (0.91 ms
- * against 0.75 ms at B1 N37810 H56 D128), which keep more memory streams in
- * flight; sage_attn_fwd uses the separate kernels.
+/* All three prepasses: the outputs of sage_quant_qk and sage_quant_v, bit
+ * for bit (same K sum, same rounding), with every byte of Q, K and V read
+ * from HBM once (the pages' producer fusions, "Sage2 Blackwell Mainloop",
+ * section "Completed P1 And P2").
+ *   - Where it applies, one cooperative kernel does all three: each of its
+ *     CTAs (two per SM) owns a fixed run of 64-token chunks of every head,
+ *     keeps its slices of a head's K and V in shared memory from the
+ *     statistics to the quantisation, and takes the heads in groups, the
+ *     statistics of one group overlapping the quantisation of the previous
+ *     one.  It applies when one CTA's slice of a head is at most 32 KB
+ *     (ceil(N/64) chunks over the CTA count, times D, at most 256:
+ *     N <= 37,888 at D = 128 and N <= 75,776 at D = 64 on 148 SMs) and the
+ *     device supports cooperative launches.  Elsewhere the separate kernels of sage_quant_qk and
+ *     sage_quant_v run instead.  sage_quant_qkv_kernels says which.
+ *   - The K mean: each channel's FP64 sum is taken from an accumulator that
+ *     the CTAs add to atomically when every partial sum of the channel is
+ *     exact in FP64 (a bound on the channel's exponent range, checked per
+ *     channel), and from the chunk partials in chunk order otherwise; both
+ *     give the chunk-order sum of the definition.
+ *   - The CTAs wait for each other's statistics with bounded waits; a wait
+ *     that runs out leaves SAGE_ERR_TIMEOUT in the status word, and the
+ *     kernel then returns.
+ *   - On one B200 the single launch is slower than the separate kernels
+ *     (1.3 ms against 0.65 ms at B1 N37810 H56 D128): its 2 x B*H steps are
+ *     synchronised across all CTAs and bound by latency.  sage_attn_fwd runs
+ *     the separate kernels.
  * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QKV, ...), 256-byte
  * aligned; concurrent calls need separate workspaces. */
 SAGE_API int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, int N, int H, int D,
                    int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
                    uint8_t* v_fp8, float* v_scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Kernel launches that sage_quant_qkv makes for this shape on the current
+ * device: 1 for the single cooperative kernel, 6 for the separate kernels; a
+ * negative SAGE_ERR_* for a shape the library refuses.  No counterpart in
+ * the pages (launch accounting). */
+SAGE_API int sage_quant_qkv_kernels(int B, int N, int H, int D);
 
 /* Fused mainloop on quantised inputs: every 64-key tile in increasing order,
  * INT8 QK^T, score scaling, online softmax, E4M3 P, two K32 FP16 PV buffers
@@ -277,7 +298,9 @@ SAGE_API int sage_get_mainloop(void);
 /* Test export for failure detection.  From the next call on, the tcgen05
  * mainloop's producer withholds K/V tile `k_tile` of every CTA (< 0: none),
  * and every bounded device wait gives up after `wait_limit_cycles` SM clock
- * cycles (<= 0: the default, about one second).  A withheld tile makes the
+ * cycles (<= 0: the default, about one second).  In the single-launch
+ * prepass (sage_quant_qkv, sage_attn_fwd) CTA 0 withholds instead its
+ * count for the K statistics of head unit b*H + h == k_tile.  A withheld tile makes the
  * waits run out: the kernel records SAGE_ERR_TIMEOUT in the status word,
  * abandons the work, frees its tensor memory and returns, leaving the
  * context usable.  Process-wide; call with (-1, 0) to restore. */

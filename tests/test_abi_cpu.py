@@ -102,9 +102,9 @@ def test_argument_errors_need_no_device(lib):
                None) == sage.SAGE_ERR_INVALID_ARG
     assert qkv(v4, v4, v4, 1, 10, 2, 64, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 100,
                None) == sage.SAGE_ERR_WORKSPACE
-    # the single-launch prepass's int work-item counter: 2^14 heads of 2^24 tokens need too many items
+    # no work-item limit beyond the common shape limits: a large problem only needs its workspace
     assert qkv(v4, v4, v4, 1, 1 << 24, 1 << 14, 128, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
-               None) == sage.SAGE_ERR_UNSUPPORTED
+               None) == sage.SAGE_ERR_WORKSPACE
     assert qkv(v4, v4, v4, 70000, 10, 1, 64, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 4096, 1 << 20,
                None) == sage.SAGE_ERR_UNSUPPORTED
     assert lib.sage_set_mainloop(7) == sage.SAGE_ERR_UNSUPPORTED

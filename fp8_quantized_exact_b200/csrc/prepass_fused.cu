@@ -8,39 +8,39 @@
 // do ("Sage2 Blackwell Mainloop", section "Completed P1 And P2").  Bytes and
 // scales equal those of the separate kernels.
 //
-// Layout of the work.  One CTA per SM (grid G <= SM count, a cooperative
-// launch, so all CTAs are resident together).  CTA i owns a fixed run of
-// 64-token chunks, [i*T64/G, (i+1)*T64/G), in every head; its slice of one
-// head is at most 64 KB.  Heads (units u = b*H + h) are taken g at a time
-// ("groups") in two passes, K with Q, then V.  At step s a CTA:
-//   1. starts the copy of the slices of step s+1 into shared memory
-//      (cp.async, three 64 KB slots);
-//   2. computes the statistics of the slices of step s (K: FP64 sums, V:
-//      absolute maxima) and publishes them with atomics, then counts itself
-//      in for each unit of the group;
-//   3. in the K pass, quantises the Q rows of its chunks (plain loads issued
-//      at the start of the step);
-//   4. waits (bounded) until all G CTAs have counted in for the group of
-//      step s-1, and quantises that group's K or V slices, which are still
-//      in shared memory.
+// Layout of the work.  A cooperative launch of G CTAs, two per SM, all
+// resident together.  CTA i owns a fixed run of 64-token chunks,
+// [i*T64/G, (i+1)*T64/G), in every head; its slice of one head's K or V is
+// at most 32 KB.  Heads (units u = b*H + h) are taken g at a time
+// ("groups") in two passes, K with Q, then V.  At step s of a CTA:
+//   1. warps 8-15 start the copies of the slices of step s+1 into one of
+//      three shared-memory slots (cp.async), and in the K pass load the Q
+//      rows of the CTA's chunks into registers;
+//   2. warps 0-7 compute the statistics of the slices of step s (K: FP64
+//      chunk sums, V: absolute maxima), publish them with atomics and count
+//      the CTA in for each unit of the group; meanwhile warps 8-15 quantise
+//      the Q rows;
+//   3. warps 0-7 wait (bounded) until all G CTAs have counted in for the
+//      group of step s-1 and form its K means or V scales;
+//   4. all warps quantise that group's K or V from the slices that are
+//      still in shared memory.
 // So K and V are read once, and the statistics of one group overlap the
 // quantisation of the previous one.
 //
 // The K mean.  The definition is the FP64 sum of the FP64 chunk partials
 // in chunk order, each partial a token-order FP64 sum, divided by N in FP64
-// and rounded once to FP32.  When every addition in that chain is exact,
-// any order and grouping of the additions gives the same bits.  A BF16 value
-// of biased exponent e is a multiple of 2^(max(e,1)-134), and its magnitude
-// is below 2^(e-126).  Take emax and emin, the largest and smallest such e
-// (emin over the nonzero values, with e taken as at least 1).  Every partial
-// sum of a channel is then a multiple of 2^(emin-134) and below
-// N * 2^(emax-126) in magnitude.  It is exactly representable in FP64 when
-// ceil(log2 N) + emax <= emin + 45.  Each CTA therefore adds its local
-// (exact) sum into an FP64 accumulator with an atomic add, and publishes
-// emax and 255 - emin with atomic maxima.  A channel that meets the bound
-// takes its mean from the accumulator.  For a channel that does not, the
-// CTAs add the chunk partials (written to k_part) in chunk order, one warp
-// per channel.  Every CTA computes the same means; CTA 0 stores them.
+// and rounded once to FP32.  The chunk partials are computed exactly so.  A
+// nonzero partial p is a multiple of 2^lo(p), its lowest set bit, and below
+// 2^(hi(p)+1) in magnitude; with lo and hi the minimum and maximum over a
+// channel's chunks, every sum of partials is a multiple of 2^lo below
+// 2^(ceil(log2 T64)+hi+1), so it is exact in FP64 when
+// ceil(log2 T64) + hi - lo <= 52.  Then any order of adding the partials
+// gives the chunk-order sum, bit for bit.  Each CTA therefore adds its
+// partials (in order) into an FP64 accumulator with an atomic add and
+// publishes hi and lo with atomic maxima; a channel within the bound takes
+// its mean from the accumulator.  For a channel outside it, the CTAs add
+// the partials (written to k_part) in chunk order, one warp per channel.
+// Every CTA computes the same means; CTA 0 stores them.
 //
 // Waits.  A CTA only waits for counts that every CTA reaches without
 // waiting on anything itself: the statistics of step s come before its wait
@@ -90,7 +90,6 @@ struct ResArgs {
 };
 
 __device__ __forceinline__ uint4 ldg16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-
 
 // Shared-memory image of a slice: token rows of D BF16 values; the 16-byte
 // piece k of row r is stored at position k ^ ((r >> 4) & 3), so that reads

@@ -12,21 +12,19 @@
 // resident together.  CTA i owns a fixed run of 64-token chunks,
 // [i*T64/G, (i+1)*T64/G), in every head; its slice of one head's K or V is
 // at most 32 KB.  Heads (units u = b*H + h) are taken g at a time
-// ("groups") in two passes, K with Q, then V.  At step s of a CTA:
-//   1. warps 8-15 start the copies of the slices of step s+1 into one of
-//      three shared-memory slots (cp.async), and in the K pass load the Q
-//      rows of the CTA's chunks into registers;
-//   2. warps 0-7 compute the statistics of the slices of step s (K: FP64
-//      chunk sums, V: absolute maxima), publish them with atomics and count
-//      the CTA in for each unit of the group; meanwhile warps 8-15 quantise
-//      the Q rows;
-//   3. warps 0-7 wait (bounded) until all G CTAs have counted in for the
-//      group of step s-1 and form its K means or V scales;
-//   4. all warps quantise that group's K or V from the slices that are
-//      still in shared memory.
+// ("groups") in two passes, K with Q, then V.  The two warpgroups of a CTA
+// form a two-stage pipeline over the steps (one group each):
+//   - warps 0-7 (statistics): wait for the slices of step s, compute their
+//     statistics (K: FP64 chunk sums, V: absolute maxima), publish them with
+//     atomics and count the CTA in; then wait (bounded) until all G CTAs
+//     have counted in for step s-1 and form its K means or V scales;
+//   - warps 8-15 (quant): copy the slices of step s+1 into one of three
+//     shared-memory slots (cp.async), quantise the Q rows of step s (K
+//     pass), then quantise K or V of step s-1 from the slices that are still
+//     resident.
 // So K and V are read once, and the statistics of one group overlap the
 // quantisation of the previous one.
-//
+
 // The K mean.  The definition is the FP64 sum of the FP64 chunk partials
 // in chunk order, each partial a token-order FP64 sum, divided by N in FP64
 // and rounded once to FP32.  The chunk partials are computed exactly so.  A
@@ -50,6 +48,7 @@
 #include <algorithm>
 
 #include "prepass_codes.cuh"
+#include "tc_prims.cuh"
 
 namespace sage {
 namespace {
@@ -483,18 +482,19 @@ __device__ void v_scales(const ResArgs& a, int grp, float* vinv_s) {
   }
 }
 
-// K: 2D threads per 64-row chunk (all chunks of a step at once) from the
-// resident slice; x' = fl32(x - km).
+// K (quant warps): 2D threads per 64-row chunk from the resident slice;
+// x' = fl32(x - km).
 template <int D>
 __device__ void k_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r, const float* kmean_s, float* red,
                         int* s_any) {
-  constexpr int SEG = D / 8, TPI = 2 * D, WPI = TPI / 32, IPP = kRThreads / TPI;
+  constexpr int SEG = D / 8, TPI = 2 * D, WPI = TPI / 32, IPP = kHalf / TPI;
   constexpr int PER = kKTile * SEG / TPI;  // 4
-  const int tt = threadIdx.x % TPI, piece = tt % SEG, col = piece * 8;
+  const int qt = threadIdx.x - kHalf;
+  const int tt = qt % TPI, piece = tt % SEG, col = piece * 8;
   uint32_t* redb = reinterpret_cast<uint32_t*>(red);
   const int items = a.g * a.cpc;
   for (int it0 = 0; it0 < items; it0 += IPP) {
-    const int item = it0 + threadIdx.x / TPI;
+    const int item = it0 + qt / TPI;
     const int i = item / a.cpc, cc = item % a.cpc;
     const int u = grp * a.g + i;
     const bool live = item < items && u < a.U && cc < r.n;
@@ -519,17 +519,17 @@ __device__ void k_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r,
     }
     // the bits of non-negative floats order as integers, NaN above inf
     const uint32_t ab = __reduce_max_sync(0xffffffffu, __float_as_uint(amax));
-    if (threadIdx.x == 0) *s_any = 0;
-    if ((threadIdx.x & 31) == 0) redb[threadIdx.x >> 5] = ab;
-    __syncthreads();
-    const uint32_t* rb = redb + (threadIdx.x / TPI) * WPI;
+    if (qt == 0) *s_any = 0;
+    if ((qt & 31) == 0) redb[qt >> 5] = ab;
+    bar_half(kBarQ);
+    const uint32_t* rb = redb + (qt / TPI) * WPI;
     uint32_t m = rb[0];
 #pragma unroll
     for (int w = 1; w < WPI; ++w) m = max(m, rb[w]);
     const bool finite = m < 0x7F800000u;
     amax = __uint_as_float(m);
     if (!finite) *s_any = 1;
-    __syncthreads();
+    bar_half(kBarQ);
     if (*s_any) {
       // NaN or inf among the rows: the amax that ignores NaN (the reference form)
       float af = 0.0f;
@@ -545,14 +545,14 @@ __device__ void k_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r,
           }
         }
       af = warp_max(af);
-      if ((threadIdx.x & 31) == 0) red[16 + (threadIdx.x >> 5)] = af;
-      __syncthreads();
-      const float* rw = red + 16 + (threadIdx.x / TPI) * WPI;
+      if ((qt & 31) == 0) red[16 + (qt >> 5)] = af;
+      bar_half(kBarQ);
+      const float* rw = red + 16 + (qt / TPI) * WPI;
       amax = rw[0];
 #pragma unroll
       for (int w = 1; w < WPI; ++w) amax = fmaxf(amax, rw[w]);
     }
-    __syncthreads();  // red is reused by the next items
+    bar_half(kBarQ);  // red is reused by the next items
     if (live) {
       const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
       const bool fast = finite && codes_fast(amax, inv);
@@ -575,7 +575,7 @@ __device__ void k_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r,
   }
 }
 
-// V: runs of 16 tokens of one channel from the resident slice converted to
+// V (quant warps): runs of 16 tokens of one channel from the resident slice converted to
 // E4M3 (token t in byte t of the channel's row) and stored as one 16-byte
 // vector; a warp covers four runs of eight channels (64 contiguous bytes
 // per channel).
@@ -583,7 +583,7 @@ template <int D>
 __device__ void v_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r, const float* vinv_s) {
   constexpr int SEG = D / 8;
   const int runs = a.g * a.cpc * 4 * D;
-  for (int idx = threadIdx.x; idx < runs; idx += kRThreads) {
+  for (int idx = threadIdx.x - kHalf; idx < runs; idx += kHalf) {
     const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
     const int cb = rest % SEG, item = rest / SEG;
     const int i = item / a.cpc, cc = item % a.cpc;
@@ -612,67 +612,117 @@ __device__ void v_quant(const ResArgs& a, int grp, const uint8_t* slot, Range r,
 // Dynamic shared memory: the slots, then the scratch.
 constexpr size_t kScratchOff = (size_t)kSlots * kSlotBytes;
 constexpr size_t kSmemBytes = kScratchOff + kMaxSliceChunkD * sizeof(double)  // sp (FP64 partials / FP32 maxima)
-                              + kMaxSliceChunkD * sizeof(float)                // mean_s (K means / V 448/amax)
+                              + 2 * kMaxSliceChunkD * sizeof(float)            // mean_buf[2] (K means / V 448/amax)
                               + kMaxSliceChunkD * sizeof(int)                  // list
                               + 64 * sizeof(float);                            // red (K: 32), redq (Q: 32)
 
-// Step st (0 <= st <= 2S): statistics of group st (K for st < S, V after)
-// and, in the K pass, the Q rows of group st; then the quantisation of
-// group st - 1 from its resident slices.
+// The two warpgroups run as a pipeline, handing over through mbarriers:
+//   statistics warps, step st: wait for the slices of step st; statistics;
+//     count in; wait (bounded) for all CTAs' counts of step st-1; its K
+//     means or V inverse scales into mean_buf[(st-1) & 1]; means_ready.
+//   quant warps, step st: copies of step st+1 into the slot that step st-2
+//     left; in the K pass the Q rows of step st; wait for means_ready of
+//     step st-1, quantise its slices; means_free.
+// Slot st % 3 is written by the copies of step st, read by the statistics of
+// step st and by the quantisation at quant step st+1, and refilled at quant
+// step st+2, after this warpgroup's own quantisation of it.
+struct Pipe {
+  uint64_t slot_full[kSlots];  // the copies of a slot have landed (256 cp.async arrivals)
+  uint64_t means_ready[2];     // mean_buf[b] holds the means of the next step to quantise
+  uint64_t means_free[2];      // the quant warps are done with mean_buf[b]
+  int abort;                   // CTA-local: a bounded wait gave up
+  int flag;                    // 0 once the statistics warps' global wait failed
+  int cnt, anyq, anyk;
+};
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kRThreads, kCtasPerSm) prepass_resident_kernel(const __grid_constant__ ResArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   double* sp = reinterpret_cast<double*>(smem + kScratchOff);
-  float* mean_s = reinterpret_cast<float*>(sp + kMaxSliceChunkD);
-  int* list = reinterpret_cast<int*>(mean_s + kMaxSliceChunkD);
+  float* mean_buf = reinterpret_cast<float*>(sp + kMaxSliceChunkD);  // [2][kMaxSliceChunkD]
+  int* list = reinterpret_cast<int*>(mean_buf + 2 * kMaxSliceChunkD);
   float* red = reinterpret_cast<float*>(list + kMaxSliceChunkD);
   uint32_t* redq = reinterpret_cast<uint32_t*>(red + 32);
-  __shared__ int s_flag, s_cnt, s_anyq, s_anyk;
+  __shared__ Pipe pp;
+  volatile int* abort_cta = &pp.abort;
 
   const Range rk = cta_range(a.T64, a.G);
   const Range rq = cta_range(a.TQ, a.G);
   const int total = 2 * a.S;
-  const bool stats_warp = threadIdx.x < kHalf;
   auto slot = [&](int st) { return smem + (size_t)(st % kSlots) * kSlotBytes; };
+  auto kind_of = [&](int st) { return st < a.S ? 0 : 1; };
 
-  if (threadIdx.x == 0) s_flag = 1;
-  issue_slices<D>(a, 0, 0, slot(0), rk);
-  cp_async_commit();
-  for (int st = 0; st <= total; ++st) {
-    if (st + 1 < total) issue_slices<D>(a, st + 1 < a.S ? 0 : 1, (st + 1) % a.S, slot(st + 1), rk);
-    cp_async_commit();
-    const bool kstep = st < a.S;
-    uint4 qx[kQPieces];
-    if (!stats_warp && kstep) q_load<D>(a, st, rq, qx);
-    cp_async_wait<1>();
-    __syncthreads();  // the slices of step st are in (every thread's copies)
-    if (stats_warp) {
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) tc::mbar_init(&pp.slot_full[i], kHalf);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&pp.means_ready[i], 1);
+      tc::mbar_init(&pp.means_free[i], 1);
+    }
+    pp.abort = 0;
+    pp.flag = 1;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (threadIdx.x < kHalf) {
+    // ------------------------------------------------- statistics warps
+    for (int st = 0; st <= total; ++st) {
       if (st < total) {
-        if (kstep) k_stats<D>(a, st, slot(st), rk, sp);
+        if (!tc::wait_bounded(&pp.slot_full[st % kSlots], (uint32_t)((st / kSlots) & 1), abort_cta, a.status, 42,
+                              a.wait_limit))
+          break;
+        if (st < a.S) k_stats<D>(a, st, slot(st), rk, sp);
         else v_stats<D>(a, st - a.S, slot(st), rk, reinterpret_cast<float*>(sp));
-        count_in(a, kstep ? 0 : 1, st % a.S);
+        count_in(a, kind_of(st), st % a.S);
       }
       if (st >= 1) {
-        const int pv = st - 1, kind = pv < a.S ? 0 : 1, grp = pv % a.S;
-        if (wait_group(a, kind, grp, &s_flag)) {
-          if (kind == 0) k_means<D>(a, grp, mean_s, list, &s_cnt);
-          else v_scales<D>(a, grp, mean_s);
+        const int pv = st - 1, kind = kind_of(pv), grp = pv % a.S, b = pv & 1;
+        const bool ok = wait_group(a, kind, grp, &pp.flag) &&
+                        tc::wait_bounded(&pp.means_free[b], (uint32_t)(((pv >> 1) & 1) ^ 1), abort_cta, a.status,
+                                         43, a.wait_limit);
+        if (ok) {
+          if (kind == 0) k_means<D>(a, grp, mean_buf + b * kMaxSliceChunkD, list, &pp.cnt);
+          else v_scales<D>(a, grp, mean_buf + b * kMaxSliceChunkD);
+        } else if (threadIdx.x == 0) {
+          pp.flag = 0;
         }
+        bar_half(kBarStats);
+        if (threadIdx.x == 0) tc::mbar_arrive(&pp.means_ready[b]);  // also on failure: the quant warps look at flag
+        if (!ok) break;
       }
-    } else if (kstep) {
-      q_quant<D>(a, st, rq, qx, redq, &s_anyq);
     }
-    __syncthreads();
-    if (!s_flag) {
-      cp_async_wait<0>();  // no copy may land after the CTA has left
-      return;
+  } else {
+    // ------------------------------------------------------ quant warps
+    issue_slices<D>(a, kind_of(0), 0, slot(0), rk);
+    cp_async_arrive_noinc(&pp.slot_full[0]);
+    for (int st = 0; st <= total; ++st) {
+      if (st + 1 < total) {
+        bar_half(kBarQ);  // every quant thread is done with the slot of step st-2
+        issue_slices<D>(a, kind_of(st + 1), (st + 1) % a.S, slot(st + 1), rk);
+        cp_async_arrive_noinc(&pp.slot_full[(st + 1) % kSlots]);
+      }
+      if (st < a.S) {
+        uint4 qx[kQPieces];
+        q_load<D>(a, st, rq, qx);
+        q_quant<D>(a, st, rq, qx, redq, &pp.anyq);
+      }
+      if (st >= 1) {
+        const int pv = st - 1, b = pv & 1;
+        const bool ok = tc::wait_bounded(&pp.means_ready[b], (uint32_t)((pv >> 1) & 1), abort_cta, a.status, 44,
+                                         a.wait_limit);
+        if (!ok || !pp.flag) break;
+        const float* mb = mean_buf + b * kMaxSliceChunkD;
+        if (pv < a.S) k_quant<D>(a, pv, slot(pv), rk, mb, red, &pp.anyk);
+        else v_quant<D>(a, pv - a.S, slot(pv), rk, mb);
+        bar_half(kBarQ);
+        if (threadIdx.x == kHalf) tc::mbar_arrive(&pp.means_free[b]);
+      }
     }
-    if (st >= 1) {
-      const int pv = st - 1;
-      if (pv < a.S) k_quant<D>(a, pv, slot(pv), rk, mean_s, red, &s_anyk);
-      else v_quant<D>(a, pv - a.S, slot(pv), rk, mean_s);
-    }
-    __syncthreads();  // slot (st - 1) % 3 is refilled at the next step
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no copy may land after the CTA has left
   }
 }
 

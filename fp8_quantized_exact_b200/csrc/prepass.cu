@@ -309,13 +309,15 @@ __global__ void __launch_bounds__(128, 8) quant_k_kernel(const uint16_t* __restr
 }
 
 // V: one 256-thread block per 128 tokens of one head.  The BF16 rows are
-// staged in shared memory with 16-byte loads; the 16-byte chunk index of a
-// row is XORed with bits 4-5 of its token, so that the column reads below
-// (four 16-token runs x eight channels per warp) fall in distinct banks.
-// Each thread then converts 16 consecutive tokens of one channel to E4M3
-// (two tokens per conversion, the earlier token in the low byte, so token t
-// is byte t of the channel's row) and writes them as one 16-byte vector; a
-// warp writes eight channels x 64 contiguous bytes.
+// copied into shared memory with cp.async (rows past N zero-filled); the
+// 16-byte piece k of row r is stored at k ^ (2 * ((r >> 4) & 3)).  Each
+// thread then takes two adjacent channels of 16 consecutive tokens: one
+// 4-byte shared load per token gives both channels, and the loads of a warp
+// (four 16-token runs x eight channel pairs over two pieces) fall in 32
+// distinct banks.  Each channel's 16 tokens are converted to E4M3 (two
+// tokens per conversion, the earlier token in the low byte, so token t is
+// byte t of the channel's row) and written as one 16-byte vector; a warp
+// writes 16 channels x 64 contiguous bytes.
 constexpr int kVTokens = 2 * kKTile;  // tokens per quant_v block
 
 template <int D>
@@ -323,56 +325,65 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict
                                                       int64_t sn, int64_t sh, int N, int H, int Nk,
                                                       const float* __restrict__ v_amax,
                                                       uint8_t* __restrict__ v8, float* __restrict__ v_scale) {
-  constexpr int SEG = D / 8;                   // 16-byte chunks per token row
-  constexpr int LOADS = kVTokens * SEG / 256;  // chunks staged per thread
-  constexpr int RUNS = D * (kVTokens / 16) / 256;  // 16-token runs converted per thread
+  constexpr int SEG = D / 8;                          // 16-byte pieces per token row
+  constexpr int COPIES = kVTokens * SEG / 256;        // pieces copied per thread
+  constexpr int RUNS = (D / 2) * (kVTokens / 16) / 256;  // (channel pair, 16-token run)s per thread
   __shared__ __align__(16) uint4 tile[kVTokens * SEG];
   // heads in the reverse of the statistics pass's order (its last rows are
   // still in L2)
   const int h = H - 1 - (int)blockIdx.y, b = (int)gridDim.z - 1 - (int)blockIdx.z;
   const int n0 = blockIdx.x * kVTokens;
   const uint16_t* vp = v + b * sb + h * sh;
-  uint4 x[LOADS];
+  const uint32_t ts0 = smem_u32(tile);
 #pragma unroll
-  for (int i = 0; i < LOADS; ++i) {
+  for (int i = 0; i < COPIES; ++i) {
     const int idx = threadIdx.x + 256 * i;
     const int r = idx / SEG, k = idx % SEG;
-    x[i] = n0 + r < N ? ldg16(vp + (int64_t)(n0 + r) * sn + k * 8) : make_uint4(0, 0, 0, 0);
+    const bool valid = n0 + r < N;
+    cp_async_16_zfill(ts0 + (uint32_t)((r * SEG + (k ^ (2 * ((r >> 4) & 3)))) * 16),
+                      valid ? vp + (int64_t)(n0 + r) * sn + k * 8 : vp, valid);
   }
-#pragma unroll
-  for (int i = 0; i < LOADS; ++i) {
-    const int idx = threadIdx.x + 256 * i;
-    const int r = idx / SEG, k = idx % SEG;
-    tile[r * SEG + (k ^ ((r >> 4) & 3))] = x[i];
-  }
+  cp_async_commit();
+  cp_async_wait<0>();
   __syncthreads();
-  const uint16_t* ts = reinterpret_cast<const uint16_t*>(tile);
+  const uint8_t* tb = reinterpret_cast<const uint8_t*>(tile);
   const float* am = v_amax + (size_t)(b * H + h) * D;
 #pragma unroll
   for (int i = 0; i < RUNS; ++i) {
     const int idx = threadIdx.x + 256 * i;
-    const int q = idx & 3, cl = (idx >> 2) & 7, rest = idx >> 5;
-    const int cb = rest % SEG, half = rest / SEG;
+    const int q = idx & 3, cp = (idx >> 2) & 7, rest = idx >> 5;
+    const int pg = rest % (SEG / 2), half = rest / (SEG / 2);
     const int t0 = half * kKTile + 16 * q;  // first token of the run; (t >> 4) & 3 == q
     if (n0 + half * kKTile >= Nk) continue;  // past the padded length
-    const int ch = cb * 8 + cl;
-    const float a = am[ch];
-    const float inv = a > 0.0f ? __fdiv_rn(448.0f, a) : 0.0f;
-    if (n0 == 0 && t0 == 0)  // the channel's scale, once per head
-      v_scale[(size_t)(b * H + h) * D + ch] = a > 0.0f ? __fdiv_rn(a, 448.0f) : 0.0f;
-    const uint16_t* col = ts + (cb ^ q) * 8 + cl;
-    uint32_t w[4];
+    const int c0 = pg * 16 + 2 * cp;        // channels c0, c0 + 1
+    const int k = c0 >> 3;                  // their piece
+    const float a0 = am[c0], a1 = am[c0 + 1];
+    const float i0 = a0 > 0.0f ? __fdiv_rn(448.0f, a0) : 0.0f;
+    const float i1 = a1 > 0.0f ? __fdiv_rn(448.0f, a1) : 0.0f;
+    if (n0 == 0 && t0 == 0) {  // the channels' scales, once per head
+      v_scale[(size_t)(b * H + h) * D + c0] = a0 > 0.0f ? __fdiv_rn(a0, 448.0f) : 0.0f;
+      v_scale[(size_t)(b * H + h) * D + c0 + 1] = a1 > 0.0f ? __fdiv_rn(a1, 448.0f) : 0.0f;
+    }
+    const uint8_t* col = tb + ((k ^ (2 * q)) << 4) + ((c0 & 7) << 1);
+    uint32_t wa[4], wc[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int t = t0 + 4 * j;
-      const uint32_t lo = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[t * D]), inv),
-                                 __fmul_rn(bf16_bits_to_f32(col[(t + 1) * D]), inv));
-      const uint32_t hi = e4m3x2(__fmul_rn(bf16_bits_to_f32(col[(t + 2) * D]), inv),
-                                 __fmul_rn(bf16_bits_to_f32(col[(t + 3) * D]), inv));
-      w[j] = a > 0.0f ? (lo | (hi << 16)) : 0u;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = *reinterpret_cast<const uint32_t*>(col + (t + e) * SEG * 16);
+      const uint32_t alo = e4m3x2(__fmul_rn(__uint_as_float(w[0] << 16), i0), __fmul_rn(__uint_as_float(w[1] << 16), i0));
+      const uint32_t ahi = e4m3x2(__fmul_rn(__uint_as_float(w[2] << 16), i0), __fmul_rn(__uint_as_float(w[3] << 16), i0));
+      const uint32_t clo = e4m3x2(__fmul_rn(__uint_as_float(w[0] & 0xFFFF0000u), i1),
+                                  __fmul_rn(__uint_as_float(w[1] & 0xFFFF0000u), i1));
+      const uint32_t chi = e4m3x2(__fmul_rn(__uint_as_float(w[2] & 0xFFFF0000u), i1),
+                                  __fmul_rn(__uint_as_float(w[3] & 0xFFFF0000u), i1));
+      wa[j] = a0 > 0.0f ? (alo | (ahi << 16)) : 0u;
+      wc[j] = a1 > 0.0f ? (clo | (chi << 16)) : 0u;
     }
-    uint8_t* dst = v8 + ((size_t)(b * H + h) * D + ch) * Nk + n0 + t0;
-    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    uint8_t* dst = v8 + ((size_t)(b * H + h) * D + c0) * Nk + n0 + t0;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    *reinterpret_cast<uint4*>(dst + Nk) = make_uint4(wc[0], wc[1], wc[2], wc[3]);
   }
 }
 

@@ -423,7 +423,7 @@ int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* ou
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
   // the separate prepass kernels: faster than the single launch on B200
-  // (0.63 against 1.1-1.3 ms at B1 N37810 H56 D128)
+  // (0.6 against 1.1 ms at B1 N37810 H56 D128)
   return fwd_body(q, k, v, out, out_stride_b, out_stride_n, out_stride_h, B, N, H, D, sm_scale, workspace,
                   workspace, false, s);
 }

@@ -184,7 +184,7 @@ SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t*
  *     that runs out leaves SAGE_ERR_TIMEOUT in the status word, and the
  *     kernel then returns.
  *   - On one B200 the single launch is slower than the separate kernels
- *     (1.1-1.3 ms against 0.63 ms at B1 N37810 H56 D128): its 2 x B*H steps
+ *     (1.1 ms against 0.6 ms at B1 N37810 H56 D128): its 2 x B*H steps
  *     are synchronised across all CTAs and bound by latency.  sage_attn_fwd runs
  *     the separate kernels.
  * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QKV, ...), 256-byte

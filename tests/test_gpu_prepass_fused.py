@@ -212,3 +212,23 @@ def test_non_finite_and_tiny_groups_take_the_reference_form(sage):
         got = q8[0, h, 32 * g:32 * g + 32]
         assert np.array_equal(got, want), (h, g)
         assert qs[0, h, g] == (np.float32(am) / np.float32(127.0) if am > 0 else 0), (h, g)
+
+
+def test_shapes_past_the_slot_fall_back_to_the_separate_kernels(sage):
+    """N = 40,000 at D = 128 is 625 chunks of 64 tokens: three per CTA over
+    296 CTAs (two per SM on 148 SMs), more than a 32 KB slot holds, so
+    sage_quant_qkv runs the six separate kernels, with their bytes and a
+    clean status."""
+    dev = torch.device("cuda:0")
+    B, N, H, D = 1, 40000, 2, 128
+    assert sage.sage_quant_qkv_kernels(B, N, H, D) == 6
+    inp = synth.custom(B, N, H, D, seed=40)
+    (q, k, v), _ = gu.to_device(inp, dev)
+    a, ws = _qkv(sage, q, k, v, dev)
+    assert sage.sage_read_device_status(ws) == sage.SAGE_OK
+    b = _separate(sage, q, k, v, dev)
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    heads = [(0, 1)]
+    _check_oracle(_logical(a, N, heads), inp, heads, N)

@@ -85,4 +85,26 @@ __device__ __forceinline__ bool codes_fast(float amax, float inv) {
   return amax <= 3.4028235e38f && inv <= 3.4028235e38f;  // false for NaN and inf
 }
 
+// ------------------------------------------------------------- K mean
+// The K mean is the FP64 sum of the FP64 chunk partials in chunk order,
+// divided by N in FP64 and rounded once to FP32.  A nonzero partial p is a
+// multiple of 2^lo(p), its lowest set bit, and below 2^(hi(p)+1) in
+// magnitude.  With lo and hi the minimum and maximum over a channel's
+// chunks, every sum of partials is a multiple of 2^lo below
+// 2^(ceil(log2 T64) + hi + 1): exact in FP64 when
+// ceil(log2 T64) + hi - lo <= 52, and then any order of the additions gives
+// the chunk-order sum bit for bit.
+constexpr int kExpBias = 1100;  // keeps kExpBias + hi and kExpBias - lo positive
+
+__device__ __forceinline__ void partial_bits(double p, int& hi, int& lo) {
+  // p is a nonzero sum of BF16 values: a normal FP64 number
+  const unsigned long long bits = (unsigned long long)__double_as_longlong(p);
+  const int e = (int)((bits >> 52) & 0x7FFu);
+  const unsigned long long sig = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+  hi = e - 1023;
+  lo = e - 1075 + __ffsll((long long)sig) - 1;
+}
+
+__device__ __forceinline__ bool partials_exact(int log2t, int hi, int lo) { return log2t + hi - lo <= 52; }
+
 }  // namespace sage

@@ -206,16 +206,6 @@ __device__ void count_in(const ResArgs& a, int kind, int grp) {
 // K also reports, per channel, floor(log2 |p|) and the exponent of the
 // lowest set bit of each nonzero chunk partial p (atomic maxima of kExpBias
 // + hi and kExpBias - lo), which the K mean's exactness test needs.
-constexpr int kExpBias = 1100;
-
-__device__ __forceinline__ void partial_bits(double p, int& hi, int& lo) {
-  // p is a nonzero sum of BF16 values: a normal FP64 number
-  const unsigned long long bits = (unsigned long long)__double_as_longlong(p);
-  const int e = (int)((bits >> 52) & 0x7FFu);
-  const unsigned long long sig = (bits & 0xFFFFFFFFFFFFFull) | (1ull << 52);
-  hi = e - 1023;
-  lo = e - 1075 + __ffsll((long long)sig) - 1;
-}
 
 template <int D>
 __device__ __noinline__ void k_stats(const ResArgs& a, int grp, const uint8_t* slot, Range r, double* sp) {
@@ -433,7 +423,7 @@ __device__ __noinline__ void k_means(const ResArgs& a, int grp, float* mean_s, i
     // every sum of partials is a multiple of 2^lo below 2^(log2t + hi + 1):
     // exact in FP64 when log2t + hi - lo <= 52, and then the accumulator
     // holds the chunk-order sum (all partials zero: +0)
-    if (lov == 0 || a.log2t + hi - (kExpBias - lov) <= 52) {
+    if (lov == 0 || partials_exact(a.log2t, hi, kExpBias - lov)) {
       mean_s[c] = lov == 0 ? 0.0f : __double2float_rn(__ddiv_rn(__ldcg(a.k_sum + at), (double)a.N));
     } else {
       list[atomicAdd(s_cnt, 1)] = c;

@@ -201,18 +201,19 @@ __device__ __forceinline__ void tmem_free(uint32_t base, uint32_t cols) {
 // >= nvalid.
 template <bool TAIL>
 __device__ __forceinline__ float tile_max(const uint32_t (&S)[64], float cs, int nvalid) {
-  int mx[32];
+  // a tree of three-input integer maxima: 64 -> 22 -> 8 -> 3 -> 1
+  int v[64];
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int a = (TAIL && 2 * j >= nvalid) ? INT_MIN : (int)S[2 * j];
-    const int b = (TAIL && 2 * j + 1 >= nvalid) ? INT_MIN : (int)S[2 * j + 1];
-    mx[j] = max(a, b);
-  }
+  for (int j = 0; j < 64; ++j) v[j] = (TAIL && j >= nvalid) ? INT_MIN : (int)S[j];
+  int a[22], b[8];
 #pragma unroll
-  for (int w = 16; w > 0; w >>= 1)
+  for (int j = 0; j < 21; ++j) a[j] = __vimax3_s32(v[3 * j], v[3 * j + 1], v[3 * j + 2]);
+  a[21] = v[63];
 #pragma unroll
-    for (int j = 0; j < w; ++j) mx[j] = max(mx[j], mx[j + w]);
-  return __fmul_rn(__int2float_rn(mx[0]), cs);
+  for (int j = 0; j < 7; ++j) b[j] = __vimax3_s32(a[3 * j], a[3 * j + 1], a[3 * j + 2]);
+  b[7] = a[21];
+  const int m = __vimax3_s32(__vimax3_s32(b[0], b[1], b[2]), __vimax3_s32(b[3], b[4], b[5]), max(b[6], b[7]));
+  return __fmul_rn(__int2float_rn(m), cs);
 }
 
 // Probabilities of 16 of a row's keys (k0..k0+15) against the running max:

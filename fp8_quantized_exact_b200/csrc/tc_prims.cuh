@@ -252,13 +252,14 @@ __device__ __forceinline__ void chunk_exp(const uint32_t (&Sc)[16], int k0, floa
 
 // The exponential pass over a tile: the scores are read again from TMEM in
 // four 16-column chunks (double-buffered), so that the registers of the max
-// pass are free.  Returns the FP32 row sum.
+// pass are free.  Returns the FP32 row sum.  The load of the first chunk into
+// A has already been issued (tmem_ld16(taddr, A)) by the caller.
 template <bool TAIL>
-__device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new, int nvalid, uint32_t (&P)[16]) {
+__device__ __forceinline__ float tile_exp_issued(uint32_t taddr, float cs, float m_new, int nvalid,
+                                                 uint32_t (&P)[16], uint32_t (&A)[16]) {
   const float nm = -m_new;
   float rs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  uint32_t A[16], Bc[16];
-  tmem_ld16(taddr, A);
+  uint32_t Bc[16];
   tmem_wait_ld16(A);
   tmem_ld16(taddr + 16, Bc);
   chunk_exp<TAIL>(A, 0, cs, nm, nvalid, rs, P);
@@ -271,6 +272,13 @@ __device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new,
   tmem_wait_ld16(Bc);
   chunk_exp<TAIL>(Bc, 48, cs, nm, nvalid, rs, P);
   return __fadd_rn(__fadd_rn(rs[0], rs[1]), __fadd_rn(rs[2], rs[3]));
+}
+
+template <bool TAIL>
+__device__ __forceinline__ float tile_exp(uint32_t taddr, float cs, float m_new, int nvalid, uint32_t (&P)[16]) {
+  uint32_t A[16];
+  tmem_ld16(taddr, A);
+  return tile_exp_issued<TAIL>(taddr, cs, m_new, nvalid, P, A);
 }
 
 // ------------------------------------------------------------- tensor maps

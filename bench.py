@@ -55,9 +55,9 @@ def parse():
     ap.add_argument("--config", default="long_fused",
                     choices=["small", "ragged", "outlier", "long_fused", "d64_batch"])
     ap.add_argument("--mainloop", default="default", choices=["default", "tcgen05", "mma_sync", "tcgen05_f32"])
-    ap.add_argument("--prepass", default="separate", choices=["separate", "qkv"],
-                    help="separate: sage_quant_qk + sage_quant_v (the kernels sage_attn_fwd runs); "
-                         "qkv: sage_quant_qkv (the single cooperative kernel where it applies)")
+    ap.add_argument("--prepass", default="auto", choices=["auto", "separate", "qkv"],
+                    help="separate: sage_quant_qk + sage_quant_v (six kernels); qkv: sage_quant_qkv (one "
+                         "streaming kernel); auto: the one sage_attn_fwd picks (qkv below 128 MiB of Q, K, V)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--e2e-heads-per-chunk", type=int, default=4)
     ap.add_argument("--e2e-one-stream", action="store_true", help="all chunks on one compute stream")
@@ -355,6 +355,8 @@ def main():
     dts = [torch.int8, torch.float32, torch.int8, torch.float32, torch.float32, torch.uint8,
            torch.float32]
     qt = {n: torch.empty(s, dtype=dt, device=dev) for (n, s), dt in zip(shp.items(), dts)}
+    if args.prepass == "auto":  # sage_attn_fwd's choice
+        args.prepass = "qkv" if 3 * B * H * N * D * 2 < (128 << 20) else "separate"
     if args.prepass == "qkv":
         ws_pre = [sage.workspace(sage.SAGE_OP_QUANT_QKV, B, N, H, D, dev)]
         pre_kernels = sage.sage_quant_qkv_kernels(B, N, H, D)
@@ -466,7 +468,7 @@ def main():
             "data": "synthetic (seeded normal BF16 stand-in for the pages' video-DiT activations)",
             "config": {"workload": f"{cfg.name}: {cfg.about}", "B": B, "N": N, "H": H, "D": D,
                        "mainloop": ml_name, "parallelism": f"{world} independent replicas",
-                       "prepass": ("single cooperative kernel" if pre_kernels == 1 else
+                       "prepass": ("single streaming kernel" if pre_kernels == 1 else
                                    f"{pre_kernels} separate kernels"),
                        "l2": "inputs 1.6 GB > 126 MB L2 (no flush needed)"
                        if cfg.name == "long_fused" else "see workload"},

@@ -171,8 +171,7 @@ def sage_quant_qkv(q, k, v, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale
 
 
 def sage_quant_qkv_kernels(B, N, H, D):
-    """Kernel launches of sage_quant_qkv for this shape on the current device
-    (1: the single cooperative kernel, 6: the separate kernels)."""
+    """Kernel launches of sage_quant_qkv for this shape (1; 0 for an empty shape)."""
     n = lib().sage_quant_qkv_kernels(B, N, H, D)
     if n < 0:
         _check(n, "sage_quant_qkv_kernels")

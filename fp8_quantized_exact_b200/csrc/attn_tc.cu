@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
       // at D = 64 the first chunk of the exponential pass is requested here,
       // so that its TMEM latency overlaps the handoff of the running max (at
       // D = 128 the extra live registers spill and the step is 9% slower)
-      uint32_t A0[16];
+      [[maybe_unused]] uint32_t A0[16];
       if constexpr (D == 64) tmem_ld16(lane_addr + cols, A0);
       // running max: m(t) = max(m(t-1), tile max), m(t-1) from the partner warp
       float m_prev = -INFINITY;

@@ -25,6 +25,23 @@ std::once_flag g_mainloop_env_once;            // SAGE_MAINLOOP is read once
 std::atomic<int> g_stall_tile{-1};             // test hook (sage_debug_set_stall)
 std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
+// Prepass implementations.  SAGE_PREPASS=separate|stream, read once, picks
+// one for every call (a measurement and test hook); without it each entry
+// point uses its own default.
+enum PrepassImpl { kPrepSeparate = 0, kPrepStream = 1 };
+std::once_flag g_prepass_env_once;
+int g_prepass_env = -1;
+void read_prepass_env() {
+  const char* e = getenv("SAGE_PREPASS");
+  if (!e) return;
+  if (!strcmp(e, "separate")) g_prepass_env = kPrepSeparate;
+  else if (!strcmp(e, "stream")) g_prepass_env = kPrepStream;
+}
+int prepass_impl(int dflt) {
+  std::call_once(g_prepass_env_once, read_prepass_env);
+  return g_prepass_env >= 0 ? g_prepass_env : dflt;
+}
+
 struct Dims {
   int B, N, H, D, Nq, Nk, G32, T64;
 };
@@ -95,7 +112,7 @@ Layout plan(int op, const Dims& d) {
   const bool all3 = op == SAGE_OP_ATTN_FWD || op == SAGE_OP_QUANT_QKV;
   if (all3 || op == SAGE_OP_QUANT_QK) L.k_part = take(bh * d.T64 * d.D * sizeof(double));
   if (all3 || op == SAGE_OP_QUANT_V) L.v_amax = take(bh * d.D * sizeof(float));
-  if (op == SAGE_OP_QUANT_QKV) L.sync = take(prepass_sync_bytes(d.B, d.H, d.D));  // single-launch prepass
+  if (all3) L.sync = take(prepass_sync_bytes(d.B, d.H, d.D));  // single-launch prepasses
   L.total = off;
   return L;
 }
@@ -124,19 +141,27 @@ FusedOut fused_out(void* ws, const Layout& L, int8_t* q8, float* qs, int8_t* k8,
   return o;
 }
 
-// The three prepasses on checked arguments into the given outputs: the
-// single-launch kernel where it applies (and `single` allows it), else the
-// separate kernels.  Both give the same bytes.
+// The three prepasses on checked arguments into the given outputs, by the
+// implementation `impl` (a PrepassImpl, unless SAGE_PREPASS overrides it).
+// Both give the same bytes.
 int prepass_all(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N, int H,
                 int D, int8_t* q8, float* qs, int8_t* k8, float* ks, float* km, uint8_t* v8, float* vs,
-                void* ws, const Layout& L, void* status, bool single, cudaStream_t s) {
+                void* ws, const Layout& L, void* status, int impl, cudaStream_t s) {
   int rc;
-  if (single && prepass_fused_fits(B, N, H, D)) {
-    rc = launch_prepass_fused(q, k, v, B, N, H, D, fused_out(ws, L, q8, qs, k8, ks, km, v8, vs, status), s);
-    if (rc != SAGE_ERR_UNSUPPORTED) return rc;
-  }
+  impl = prepass_impl(impl);
+  if (impl == kPrepStream)
+    return launch_prepass_stream(q, k, v, B, N, H, D, fused_out(ws, L, q8, qs, k8, ks, km, v8, vs, status), s);
   if ((rc = launch_prepass_qk(q, k, B, N, H, D, q8, qs, k8, ks, km, at<double>(ws, L.k_part), s))) return rc;
   return launch_prepass_v(v, B, N, H, D, v8, vs, at<float>(ws, L.v_amax), s);
+}
+
+// The streaming single launch below about the L2 size of Q, K and V, where
+// the six separate launches' fixed cost dominates; the separate kernels
+// above it, where they stream faster (measured on B200: 0.016 against
+// 0.060 ms at B1 N256 H2 D128, 0.24 against 0.18 ms at B2 N8192 H32 D128).
+int default_prepass(int B, int N, int H, int D) {
+  const double bytes = 3.0 * B * H * (double)N * D * 2.0;
+  return bytes < (double)(128u << 20) ? kPrepStream : kPrepSeparate;
 }
 
 int clear_status(void* ws, cudaStream_t s) {
@@ -233,7 +258,7 @@ bool device_memory(const void* p) {
 // callers clear).
 int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, void* out,
              int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N, int H, int D,
-             float sm_scale, void* workspace, void* status, bool single_prepass, cudaStream_t s) {
+             float sm_scale, void* workspace, void* status, int prepass, cudaStream_t s) {
   int rc;
   const Dims d = make_dims(B, N, H, D);
   const Layout L = plan(SAGE_OP_ATTN_FWD, d);
@@ -244,7 +269,7 @@ int fwd_body(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_b
   float* km = at<float>(workspace, L.k_mean);
   uint8_t* v8 = at<uint8_t>(workspace, L.v8);
   float* vs = at<float>(workspace, L.v_scale);
-  if ((rc = prepass_all(q, k, v, B, N, H, D, q8, qs, k8, ks, km, v8, vs, workspace, L, status, single_prepass, s)))
+  if ((rc = prepass_all(q, k, v, B, N, H, D, q8, qs, k8, ks, km, v8, vs, workspace, L, status, prepass, s)))
     return rc;
   return run_mainloop(make_params(d, q8, qs, k8, ks, v8, vs, out, out_stride_b, out_stride_n,
                                   out_stride_h, sm_scale, status),
@@ -377,14 +402,14 @@ int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
   return prepass_all(q, k, v, B, N, H, D, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale, workspace, L,
-                     workspace, true, s);
+                     workspace, kPrepStream, s);
 }
 
 int sage_quant_qkv_kernels(int B, int N, int H, int D) {
   const int rc = check_dims(B, N, H, D);
   if (rc) return rc;
   if (empty(B, N, H)) return 0;
-  return prepass_fused_fits(B, N, H, D) ? 1 : 6;
+  return 1;
 }
 
 int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, const int8_t* k_i8,
@@ -422,10 +447,8 @@ int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* ou
   if ((rc = check_ws(workspace, workspace_bytes, L.total))) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if ((rc = clear_status(workspace, s))) return rc;
-  // the separate prepass kernels: faster than the single launch on B200
-  // (0.6 against 1.1 ms at B1 N37810 H56 D128)
   return fwd_body(q, k, v, out, out_stride_b, out_stride_n, out_stride_h, B, N, H, D, sm_scale, workspace,
-                  workspace, false, s);
+                  workspace, default_prepass(B, N, H, D), s);
 }
 
 int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_bf16 v_host,
@@ -496,11 +519,13 @@ int sage_attn_fwd_host(sage_view_bf16 q_host, sage_view_bf16 k_host, sage_view_b
       cv[i].data = static_cast<const uint16_t*>(dv[i]->data) + (int64_t)h0 * dv[i]->stride_h;
     }
     void* co = static_cast<uint16_t*>(out_dev) + (int64_t)h0 * out_stride_h;
-    // the separate prepass kernels: chunks of a few heads on two streams,
-    // overlapping other chunks' mainloops (a cooperative launch would
-    // contend with those for co-residency)
+    // the chunk's prepass by the rule of sage_attn_fwd (a chunk of a few
+    // heads is small enough for the single launch up to long sequences;
+    // measured on B200 with host buffers: 47.99 against 48.10 ms at B1
+    // N37810 H56 D128 in chunks of four heads, 0.071 against 0.099 ms at B1
+    // N256 H2 D128)
     if ((rc = fwd_body(cv[0], cv[1], cv[2], co, out_stride_b, out_stride_n, out_stride_h, B, N, h1 - h0, D,
-                       sm_scale, wsc, workspace, false, sc)))
+                       sm_scale, wsc, workspace, default_prepass(B, N, h1 - h0, D), sc)))
       return rc;
     if (!ok(cudaEventRecord(e_comp, sc)) || !ok(cudaStreamWaitEvent(s_out, e_comp, 0))) return SAGE_ERR_CUDA;
     if ((rc = copy_heads(out_host, out_dev, out_stride_b, out_stride_n, out_stride_h, B, N, D, h0, h1,

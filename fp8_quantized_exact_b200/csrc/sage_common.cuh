@@ -134,13 +134,11 @@ int launch_norm_rope_qk(const NormRopeIn& in, const sage_view_bf16& q, const sag
                         cudaStream_t s);
 void launch_reduce_k_mean(int BH, int N, int D, int T64, const double* k_part, float* k_mean, cudaStream_t s);
 // Bytes of the single-launch prepass's zeroed scratch (statistics
-// accumulators and arrival counters).
+// accumulators, counters and flags).
 size_t prepass_sync_bytes(int B, int H, int D);
-// true when the single-launch prepass applies to the shape on the current
-// device (cooperative launch, one CTA's slice of a head within 64 KB)
-bool prepass_fused_fits(int B, int N, int H, int D);
-int launch_prepass_fused(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
-                         int H, int D, const FusedOut& o, cudaStream_t s);
+// The single-launch (streaming) prepass, for any shape the separate kernels take.
+int launch_prepass_stream(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
+                          int H, int D, const FusedOut& o, cudaStream_t s);
 // k_part: B*H*T64*D doubles of scratch; v_amax: B*H*D floats (scratch, cleared by the launch)
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,

@@ -162,41 +162,35 @@ SAGE_API int sage_quant_v(sage_view_bf16 v, int B, int N, int H, int D, uint8_t*
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* All three prepasses: the outputs of sage_quant_qk and sage_quant_v, bit
- * for bit (same K sum, same rounding), with every byte of Q, K and V read
- * from HBM once (the pages' producer fusions, "Sage2 Blackwell Mainloop",
- * section "Completed P1 And P2").
- *   - Where it applies, one cooperative kernel does all three: each of its
- *     CTAs (two per SM) owns a fixed run of 64-token chunks of every head,
- *     keeps its slices of a head's K and V in shared memory from the
- *     statistics to the quantisation, and takes the heads in groups, the
- *     statistics of one group overlapping the quantisation of the previous
- *     one.  It applies when one CTA's slice of a head is at most 32 KB
- *     (ceil(N/64) chunks over the CTA count, times D, at most 256:
- *     N <= 37,888 at D = 128 and N <= 75,776 at D = 64 on 148 SMs) and the
- *     device supports cooperative launches.  Elsewhere the separate kernels of sage_quant_qk and
- *     sage_quant_v run instead.  sage_quant_qkv_kernels says which.
+ * for bit (same K sum, same rounding), in one kernel launch (after a memset
+ * of its scratch) in which K and V are read from HBM about once (the pages'
+ * producer fusions, "Sage2 Blackwell Mainloop", section "Completed P1 And
+ * P2").
+ *   - The work is a list of 64-token tiles of one head: K statistics, V
+ *     statistics, Q codes, then, a few heads later in the list, the K and V
+ *     codes of the head.  Persistent CTAs take the tiles in list order, so
+ *     a head's codes re-read its K and V while they are still in L2.
  *   - The K mean: each channel's FP64 sum is taken from an accumulator that
- *     the CTAs add to atomically when every partial sum of the channel is
+ *     the tiles add to atomically when every partial sum of the channel is
  *     exact in FP64 (a bound on the channel's exponent range, checked per
  *     channel), and from the chunk partials in chunk order otherwise; both
  *     give the chunk-order sum of the definition.
- *   - The CTAs wait for each other's statistics with bounded waits; a wait
- *     that runs out leaves SAGE_ERR_TIMEOUT in the status word, and the
- *     kernel then returns.
- *   - On one B200 the single launch is slower than the separate kernels
- *     (1.1 ms against 0.6 ms at B1 N37810 H56 D128): its 2 x B*H steps
- *     are synchronised across all CTAs and bound by latency.  sage_attn_fwd runs
- *     the separate kernels.
+ *   - A head's code tiles wait (bounded) until all of its statistics tiles
+ *     are counted in; a wait that runs out leaves SAGE_ERR_TIMEOUT in the
+ *     status word, and the kernel then returns.
+ *   - Any shape the separate kernels take.  On one B200 it is faster than
+ *     the six separate launches up to about 128 MB of Q, K and V (0.016
+ *     against 0.060 ms at B1 N256 H2 D128) and slower above (0.77 against
+ *     0.59 ms at B1 N37810 H56 D128); sage_attn_fwd picks by that size.
  * Workspace: sage_workspace_bytes(SAGE_OP_QUANT_QKV, ...), 256-byte
  * aligned; concurrent calls need separate workspaces. */
 SAGE_API int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, int N, int H, int D,
                    int8_t* q_i8, float* q_scale, int8_t* k_i8, float* k_scale, float* k_mean,
                    uint8_t* v_fp8, float* v_scale, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Kernel launches that sage_quant_qkv makes for this shape on the current
- * device: 1 for the single cooperative kernel, 6 for the separate kernels; a
- * negative SAGE_ERR_* for a shape the library refuses.  No counterpart in
- * the pages (launch accounting). */
+/* Kernel launches that sage_quant_qkv makes for this shape: 1 (0 for an
+ * empty shape); a negative SAGE_ERR_* for a shape the library refuses.  No
+ * counterpart in the pages (launch accounting). */
 SAGE_API int sage_quant_qkv_kernels(int B, int N, int H, int D);
 
 /* Fused mainloop on quantised inputs: every 64-key tile in increasing order,
@@ -213,10 +207,12 @@ SAGE_API int sage_attn_from_quant(const int8_t* q_i8, const float* q_scale, cons
                          int64_t out_stride_h, int B, int N, int H, int D, float sm_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
-/* The whole path: both prepasses (the separate kernels of sage_quant_qk and
- * sage_quant_v; quantised tensors kept in the workspace) then the fused
- * mainloop.  Workspace: sage_workspace_bytes(
- * SAGE_OP_ATTN_FWD, ...) bytes, 256-byte aligned. */
+/* The whole path: the three prepasses (below about 128 MB of Q, K and V the
+ * single launch of sage_quant_qkv, above it the separate kernels of
+ * sage_quant_qk and sage_quant_v, whichever is faster there; the same bytes
+ * either way; quantised tensors kept in the workspace) then the fused
+ * mainloop.  Workspace: sage_workspace_bytes(SAGE_OP_ATTN_FWD, ...) bytes,
+ * 256-byte aligned. */
 SAGE_API int sage_attn_fwd(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, void* out,
                   int64_t out_stride_b, int64_t out_stride_n, int64_t out_stride_h, int B, int N,
                   int H, int D, float sm_scale, void* workspace, size_t workspace_bytes,
@@ -299,8 +295,9 @@ SAGE_API int sage_get_mainloop(void);
  * mainloop's producer withholds K/V tile `k_tile` of every CTA (< 0: none),
  * and every bounded device wait gives up after `wait_limit_cycles` SM clock
  * cycles (<= 0: the default, about one second).  In the single-launch
- * prepass (sage_quant_qkv, sage_attn_fwd) CTA 0 withholds instead its
- * count for the K statistics of head unit b*H + h == k_tile.  A withheld tile makes the
+ * prepass (sage_quant_qkv, and sage_attn_fwd where it uses it) the first K
+ * statistics tile of head unit b*H + h == k_tile is never counted in
+ * instead (wait site 45).  A withheld tile makes the
  * waits run out: the kernel records SAGE_ERR_TIMEOUT in the status word,
  * abandons the work, frees its tensor memory and returns, leaving the
  * context usable.  Process-wide; call with (-1, 0) to restore. */

@@ -1,12 +1,13 @@
-"""The single-launch prepass (sage_quant_qkv) at the workload sizes, on its
-two K-mean paths, and its bounded waits.
+"""The single-launch (streaming) prepass, sage_quant_qkv, at the workload
+sizes, on its two K-mean paths, and its bounded waits.
 
 Its outputs must equal those of the separate kernels (sage_quant_qk +
 sage_quant_v) byte for byte, and the oracle's on sampled heads.  The K mean
 is taken from an atomic FP64 accumulator for channels whose exponent range
 makes every partial sum exact, and from the chunk partials in chunk order
-otherwise; a planted cancellation makes the chunk order matter, so only the
-second path gives the oracle's value there.  Groups holding NaN, inf or
+otherwise (formed once per head by the K code tile that claims them); a
+planted cancellation makes the chunk order matter, so only the second path
+gives the oracle's value there.  Groups holding NaN, inf or
 only tiny values take the reference form of the INT8 codes (conversion and
 clamp) instead of the fast rounding; both forms are checked."""
 import numpy as np
@@ -82,8 +83,9 @@ def _check_oracle(got, inp, heads, N):
 @pytest.mark.parametrize("cfg", ["outlier", "long_fused", "d64_batch"])
 def test_single_launch_at_workload_sizes(sage, cfg):
     """The B2 N8192 H32, B1 N37810 H56 (fused projection strides) and B4
-    N16384 H24 D64 workloads: one cooperative launch, the separate kernels'
-    bytes, and the oracle's bytes on three sampled heads."""
+    N16384 H24 D64 workloads (the work list taken four tiles at a time): one
+    launch, the separate kernels' bytes, and the oracle's bytes on three
+    sampled heads."""
     dev = torch.device("cuda:0")
     c = synth.CONFIGS[cfg]
     assert sage.sage_quant_qkv_kernels(c.B, c.N, c.H, c.D) == 1
@@ -138,10 +140,11 @@ def test_chunk_order_path_for_channels_off_the_bound(sage):
 
 
 def test_withheld_count_times_out_and_the_next_call_is_right(sage):
-    """CTA 0 withholds its K count for head 2 (the test hook): every CTA's
-    wait for that head runs out after about 1 ms, the status word says
-    SAGE_ERR_TIMEOUT (wait site 40), the kernel returns, and the next call
-    on the same context writes the separate kernels' bytes."""
+    """The first K statistics tile of head 2 is never counted in (the test
+    hook): the waits of that head's K code tiles run out after about 1 ms,
+    the status word says SAGE_ERR_TIMEOUT (wait site 45), the kernel
+    returns, and the next call on the same context writes the separate
+    kernels' bytes."""
     dev = torch.device("cuda:0")
     B, N, H, D = 1, 1000, 4, 128
     assert sage.sage_quant_qkv_kernels(B, N, H, D) == 1
@@ -154,7 +157,7 @@ def test_withheld_count_times_out_and_the_next_call_is_right(sage):
         code, where, block = ws[:12].view(torch.int32).tolist()
     finally:
         sage.sage_debug_set_stall(-1, 0)
-    assert st == sage.SAGE_ERR_TIMEOUT and where == 40, (st, where, block)
+    assert st == sage.SAGE_ERR_TIMEOUT and where == 45, (st, where, block)
     a, ws = _qkv(sage, q, k, v, dev)
     assert sage.sage_read_device_status(ws) == sage.SAGE_OK
     b = _separate(sage, q, k, v, dev)
@@ -173,7 +176,7 @@ def _ref_codes(x, inv):
 
 def test_non_finite_and_tiny_groups_take_the_reference_form(sage):
     """NaN and inf in some Q rows and K/V tokens, and a head whose Q and K
-    values are all tiny (inv = 127/amax overflows): the single-launch and
+    values are all tiny (inv = 127/amax overflows): the single launch and
     the separate kernels write the same bytes, and Q codes of those groups
     equal the reference form."""
     dev = torch.device("cuda:0")
@@ -214,14 +217,14 @@ def test_non_finite_and_tiny_groups_take_the_reference_form(sage):
         assert qs[0, h, g] == (np.float32(am) / np.float32(127.0) if am > 0 else 0), (h, g)
 
 
-def test_shapes_past_the_slot_fall_back_to_the_separate_kernels(sage):
-    """N = 40,000 at D = 128 is 625 chunks of 64 tokens: three per CTA over
-    296 CTAs (two per SM on 148 SMs), more than a 32 KB slot holds, so
-    sage_quant_qkv runs the six separate kernels, with their bytes and a
-    clean status."""
+def test_long_heads_take_one_launch(sage):
+    """N = 40,000 at D = 128 (625 chunks of 64 tokens per head, past what a
+    scheme that keeps a head's slices on chip would hold): still one launch,
+    the separate kernels' bytes, the oracle's on a sampled head, and a clean
+    status."""
     dev = torch.device("cuda:0")
     B, N, H, D = 1, 40000, 2, 128
-    assert sage.sage_quant_qkv_kernels(B, N, H, D) == 6
+    assert sage.sage_quant_qkv_kernels(B, N, H, D) == 1
     inp = synth.custom(B, N, H, D, seed=40)
     (q, k, v), _ = gu.to_device(inp, dev)
     a, ws = _qkv(sage, q, k, v, dev)

@@ -45,7 +45,8 @@ EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_
            "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
            "sage_strerror", "sage_set_mainloop", "sage_get_mainloop", "sage_debug_qk_s32",
-           "sage_attn_fwd_noalloc", "sage_noalloc_read_status", "sage_debug_set_stall", "sage_attn_fwd_host")
+           "sage_attn_fwd_noalloc", "sage_noalloc_read_status", "sage_debug_set_stall", "sage_attn_fwd_host",
+           "sage_debug_prepass_list")
 SAGE_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -97,6 +98,7 @@ def lib():
             "sage_attn_fwd_noalloc": [V, V, V, P, L64, L64, L64, I, I, I, I, ctypes.c_float, P],
             "sage_noalloc_read_status": [P],
             "sage_debug_set_stall": [I, ctypes.c_longlong],
+            "sage_debug_prepass_list": [I, I, I, I, I, P, ctypes.c_longlong, P],
             "sage_attn_fwd_host": [V, V, V, V, V, V, P, P, L64, L64, L64, I, I, I, I, ctypes.c_float, I, P, SZ,
                                    P, P, P, P, P, P, P],
         }
@@ -303,6 +305,18 @@ def sage_get_mainloop() -> int:
 
 def sage_debug_set_stall(k_tile: int, wait_limit_cycles: int = 0):
     _check(lib().sage_debug_set_stall(int(k_tile), int(wait_limit_cycles)), "sage_debug_set_stall")
+
+
+def sage_debug_prepass_list(B: int, N: int, H: int, D: int, grid: int):
+    """The single-launch prepass's work list on the host: (lag, int32 array of
+    (kind, head unit, 64-token tile) rows in list order)."""
+    import numpy as np
+    n = 5 * B * H * (-(-N // 128)) * 2
+    items = np.zeros((n, 3), dtype=np.int32)
+    lag = ctypes.c_int(0)
+    _check(lib().sage_debug_prepass_list(B, N, H, D, grid, ctypes.byref(lag), n, items.ctypes.data),
+           "sage_debug_prepass_list")
+    return lag.value, items
 
 
 def sage_debug_qk_s32(q_i8, q_scale, k_i8, k_scale, v_fp8, v_scale, B, N, H, D, b, h, q_tile, k_tile, s_out,

@@ -90,12 +90,14 @@ struct Item {
   int kind, u, part;
 };
 
-// Item j of the list (see the header comment for the order).
-__device__ __forceinline__ Item item_at(const StreamArgs& a, long long j) {
-  const long long seg = j / a.I, U = a.U, R = a.R;
+// Item j of the list of U heads, I tiles per kind and head, lag R (see the
+// header comment for the order).  Host and device: the host export of the
+// list is what the tests check.
+__host__ __device__ __forceinline__ Item item_at(long long U, long long I, long long R, long long j) {
+  const long long seg = j / I;
   Item it;
-  it.part = (int)(j - seg * a.I);
-  if (seg < 3 * std::min(R, U)) {
+  it.part = (int)(j - seg * I);
+  if (seg < 3 * (R < U ? R : U)) {
     it.kind = (int)(seg % 3);
     it.u = (int)(seg / 3);
   } else if (R < U && seg < 3 * R + 5 * (U - R)) {
@@ -564,7 +566,7 @@ __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) prepass_stream_kernel(
   while (j >= 0 && j < a.total) {
     long long jn = -1;
     if (threadIdx.x == 0 && left == 1) jn = take(a);  // used after this item
-    if (threadIdx.x == 0) s_it = item_at(a, j);
+    if (threadIdx.x == 0) s_it = item_at(a.U, a.I, a.R, j);
     __syncthreads();
     const Item it = s_it;
     const int b = it.u / a.H, h = it.u % a.H;
@@ -689,6 +691,20 @@ int stream(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf1
 }
 
 }  // namespace
+
+int prepass_stream_list(int B, int N, int H, int grid, int* lag, long long n, int* items) {
+  const int U = B * H, I = ceil_div(N, kQTile) * kQTile / kTok;
+  if (5LL * U * I != n || grid <= 0) return SAGE_ERR_INVALID_ARG;
+  const int R = pick_lag(U, I, grid);
+  if (lag) *lag = R;
+  for (long long j = 0; j < n; ++j) {
+    const Item it = item_at(U, I, R, j);
+    items[3 * j] = it.kind;
+    items[3 * j + 1] = it.u;
+    items[3 * j + 2] = it.part;
+  }
+  return SAGE_OK;
+}
 
 size_t prepass_sync_bytes(int B, int H, int D) {
   // per channel: an FP64 sum and three ints; per head: four ints (counts and

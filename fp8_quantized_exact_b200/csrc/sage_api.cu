@@ -570,6 +570,14 @@ int sage_set_mainloop(int which) {
 
 int sage_get_mainloop(void) { return resolved_mainloop(); }
 
+int sage_debug_prepass_list(int B, int N, int H, int D, int grid, int* lag, long long n_items, int* items) {
+  const int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return n_items == 0 ? SAGE_OK : SAGE_ERR_INVALID_ARG;
+  if (!items) return SAGE_ERR_INVALID_ARG;
+  return prepass_stream_list(B, N, H, grid, lag, n_items, items);
+}
+
 int sage_debug_set_stall(int k_tile, long long wait_limit_cycles) {
   g_stall_tile.store(k_tile < 0 ? -1 : k_tile);
   g_wait_limit.store(wait_limit_cycles > 0 ? wait_limit_cycles : kDefaultWaitLimit);

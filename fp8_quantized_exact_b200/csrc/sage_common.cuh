@@ -139,6 +139,9 @@ size_t prepass_sync_bytes(int B, int H, int D);
 // The single-launch (streaming) prepass, for any shape the separate kernels take.
 int launch_prepass_stream(const sage_view_bf16& q, const sage_view_bf16& k, const sage_view_bf16& v, int B, int N,
                           int H, int D, const FusedOut& o, cudaStream_t s);
+// Its work list for `grid` CTAs, on the host: (kind, head, tile) triples of
+// all n items, and the lag in heads.
+int prepass_stream_list(int B, int N, int H, int grid, int* lag, long long n, int* items);
 // k_part: B*H*T64*D doubles of scratch; v_amax: B*H*D floats (scratch, cleared by the launch)
 int launch_prepass_qk(const sage_view_bf16& q, const sage_view_bf16& k, int B, int N, int H, int D,
                       int8_t* q8, float* q_scale, int8_t* k8, float* k_scale, float* k_mean,

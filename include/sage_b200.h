@@ -303,6 +303,17 @@ SAGE_API int sage_get_mainloop(void);
  * context usable.  Process-wide; call with (-1, 0) to restore. */
 SAGE_API int sage_debug_set_stall(int k_tile, long long wait_limit_cycles);
 
+/* Test export, host only (no device is touched): the work list of the
+ * single-launch prepass (sage_quant_qkv) for this shape and `grid` CTAs.
+ * Writes n_items = 5 * B * H * ceil(N/128) * 2 triples (kind, head unit
+ * b*H + h, 64-token tile) to `items` in list order, kind 0 K statistics,
+ * 1 V statistics, 2 Q codes, 3 K codes, 4 V codes, and the lag in heads to
+ * `lag` (may be NULL).  The kernel's bounded waits all end because each
+ * tile appears once and every head's statistics come before its codes; a
+ * test checks both here.  SAGE_ERR_INVALID_ARG for a wrong n_items, grid <= 0
+ * or a NULL `items`. */
+SAGE_API int sage_debug_prepass_list(int B, int N, int H, int D, int grid, int* lag, long long n_items, int* items);
+
 /* Size of the fixed device array behind sage_attn_fwd_noalloc (64 MiB). */
 #define SAGE_NOALLOC_SCRATCH_BYTES (64u << 20)
 

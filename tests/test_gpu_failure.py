@@ -37,7 +37,9 @@ def test_withheld_tile_times_out_and_context_survives():
     finally:
         sage.sage_debug_set_stall(-1, 0)
     assert st == sage.SAGE_ERR_TIMEOUT and code == st, (st, where, block)
-    assert where > 0 and 0 <= block < (N + 127) // 128 * H * B
+    # a wait of the mainloop gave up (the single-launch prepass, which this
+    # shape runs, has sites 45-47 and no head unit 3 to withhold here)
+    assert 0 < where < 40 and 0 <= block < (N + 127) // 128 * H * B
     # the context is still usable and the next call is correct
     out2, _ = gu.run_fwd(sage, q, k, v, sage.SAGE_MAINLOOP_TCGEN05)
     qz = oracle.quantize(inp.q, inp.k, inp.v)

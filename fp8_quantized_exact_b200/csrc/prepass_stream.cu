@@ -16,20 +16,22 @@
 //   QQ  Q codes and scales (one 64-row block, two 32-row groups);
 //   CK  K codes and scale of x - mean (one 64-row block);
 //   CV  V codes (E4M3, transposed into channel rows).
-// CTAs take items in list order from a global counter.  Round r of the list
-// holds SK(r), SV(r), QQ(r) and, R heads behind, CK(r-R), CV(r-R).  A CTA
-// counts a finished SK (SV) item in for its head with a release (a fence and
-// a reduction), deferred until the loads of its next item are under way so
-// that the fence's wait overlaps them.  A CK (CV) item waits (bounded) until
-// all of its head's SK (SV) items are counted in and forms the K means (V
-// scales) it needs from the accumulated statistics.  A CTA only ever waits
-// for items that come earlier in the list, which running CTAs have already
-// taken and count in before their next wait, and SK, SV and QQ items wait
-// for nothing, so every wait ends.  The host picks R
-// so that about two grids' worth of items lie between a head's statistics
-// and its codes: by then the statistics are done, and R heads of Q, K and V
-// (a few tens of MB at the sizes used here, against 126 MB of L2) have
-// passed through L2 since the head's K and V were read.
+// Persistent CTAs take items in list order from a global counter, one at a
+// time or four consecutive ones when every CTA has many.  Round r of the
+// list holds SK(r), SV(r), QQ(r) and, R heads behind, CK(r-R), CV(r-R).  A
+// CTA counts a finished SK (SV) item in for its head with a release (a fence
+// and a reduction), deferred until the loads of its next item are under way
+// so that the fence's wait overlaps them.  A CK (CV) item waits (bounded)
+// until all of its head's SK (SV) items are counted in and forms the K means
+// (reads the V amax) itself from the accumulated statistics; the CTA keeps
+// them for its next items of the same head.  A CTA only ever waits for items
+// that come earlier in the list, which running CTAs have already taken and
+// count in before their next wait, and SK, SV and QQ items wait for nothing,
+// so every wait ends.  The host picks R so that about two grids' worth of
+// items lie between a head's statistics and its codes: by then the
+// statistics are done, and R heads of Q, K and V (a few tens of MB at the
+// sizes used here, against 126 MB of L2) have passed through L2 since the
+// head's K and V were read.
 //
 // The K mean is the FP64 sum of the FP64 chunk partials in chunk order,
 // divided by N in FP64 and rounded once to FP32.  A nonzero partial p is a

@@ -139,6 +139,43 @@ def test_chunk_order_path_for_channels_off_the_bound(sage):
     assert np.array_equal(km, qz.k_mean)
 
 
+def test_chunk_order_path_with_the_list_taken_in_batches(sage):
+    """The planted cancellation of the test above in two heads of a shape
+    long enough that CTAs take the work list four tiles at a time (B1
+    N46000 H4 D128: 14,400 tiles, at least 16 per CTA of a 148 x 6 grid).
+    Both heads' channels fail the bound, so their first K code tiles claim
+    the chunk-order sums and the head's other code tiles, on other CTAs,
+    wait for them; a CTA keeps the means for its next tiles of the head."""
+    dev = torch.device("cuda:0")
+    B, N, H, D = 1, 46000, 4, 128
+    inp = synth.custom(B, N, H, D, seed=91)
+    kk = inp.k
+
+    def bf16(x):
+        return np.float32(x).view(np.uint32) >> 16
+
+    T64 = -(-N // 64)
+    for h, ch in ((1, 5), (3, 77)):
+        kk[0, :, h, ch] = 0
+        kk[0, 3, h, ch] = bf16(2.0 ** 30)
+        kk[0, 64 + 9, h, ch] = bf16(-(2.0 ** 30))
+        for c in range(2, T64):
+            kk[0, 64 * c + (c % 17), h, ch] = bf16(2.0 ** -30) if 64 * c + (c % 17) < N else 0
+    (q, k, v), _ = gu.to_device(inp, dev)
+    a, ws = _qkv(sage, q, k, v, dev)
+    assert sage.sage_read_device_status(ws) == sage.SAGE_OK
+    km = a["k_mean"].cpu().numpy()
+    n_small = sum(1 for c in range(2, T64) if 64 * c + (c % 17) < N)
+    for h, ch in ((1, 5), (3, 77)):
+        assert km[0, h, ch] == np.float32(n_small * 2.0 ** -30 / N), (h, km[0, h, ch])
+    b = _separate(sage, q, k, v, dev)
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    heads = [(0, 1), (0, 3)]
+    _check_oracle(_logical(a, N, heads), inp, heads, N)
+
+
 def test_withheld_count_times_out_and_the_next_call_is_right(sage):
     """The first K statistics tile of head 2 is never counted in (the test
     hook): the waits of that head's K code tiles run out after about 1 ms,

@@ -176,6 +176,25 @@ def test_chunk_order_path_with_the_list_taken_in_batches(sage):
     _check_oracle(_logical(a, N, heads), inp, heads, N)
 
 
+def test_many_short_heads(sage):
+    """B24 N100 H64 D64: 1,536 heads of two 64-token tiles each.  The list
+    is taken four tiles at a time (15,360 tiles) and the lag is large (about
+    180 heads between a head's statistics and its codes): the separate
+    kernels' bytes, and the oracle's on two sampled heads."""
+    dev = torch.device("cuda:0")
+    B, N, H, D = 24, 100, 64, 64
+    inp = synth.custom(B, N, H, D, seed=24)
+    (q, k, v), _ = gu.to_device(inp, dev)
+    a, ws = _qkv(sage, q, k, v, dev)
+    assert sage.sage_read_device_status(ws) == sage.SAGE_OK
+    b = _separate(sage, q, k, v, dev)
+    torch.cuda.synchronize()
+    for n in a:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    heads = [(0, 0), (B - 1, H - 1)]
+    _check_oracle(_logical(a, N, heads), inp, heads, N)
+
+
 def test_withheld_count_times_out_and_the_next_call_is_right(sage):
     """The first K statistics tile of head 2 is never counted in (the test
     hook): the waits of that head's K code tiles run out after about 1 ms,

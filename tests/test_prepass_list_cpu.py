@@ -10,7 +10,7 @@ import pytest
 import fp8_quantized_exact_b200 as sage
 
 SHAPES = [(1, 256, 2, 128), (1, 1000, 8, 128), (2, 8192, 32, 128), (1, 37810, 56, 128), (4, 16384, 24, 64),
-          (1, 1, 1, 64), (3, 65, 5, 128), (1, 4000, 1, 64)]
+          (1, 1, 1, 64), (3, 65, 5, 128), (1, 4000, 1, 64), (24, 100, 64, 64)]
 
 
 @pytest.fixture(scope="module")

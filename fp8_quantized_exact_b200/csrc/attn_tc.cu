@@ -147,6 +147,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // Launched as a programmatic dependent of the prepass: the set-up above
+  // overlaps its last CTAs; nothing the prepass writes is read before this
+  // returns (the prepass grid complete, its writes visible).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp >= kSoftWarp0 && warp < kOutWarp0) {
     // ------------------------------------------------ QK / softmax owners
@@ -441,9 +445,20 @@ int launch_tc(const AttnParams& p, cudaStream_t s) {
   const size_t smem = smem_bytes<D>();
   if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  const dim3 grid = DBG ? dim3(1, 1, 1) : dim3(p.Nq / kQTile, p.H, p.B);
-  fn<<<grid, kThreadsTC, smem, s>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = DBG ? dim3(1, 1, 1) : dim3(p.Nq / kQTile, p.H, p.B);
+  cfg.blockDim = dim3(kThreadsTC);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  // programmatic dependent launch: the CTAs may start while the previous
+  // kernel of the stream drains, once every CTA of that kernel has signalled
+  // (the prepass kernels do at their start; others at their end)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, mq, mk, mv, p) == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
 }  // namespace

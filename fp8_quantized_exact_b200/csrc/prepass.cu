@@ -329,6 +329,9 @@ __global__ void __launch_bounds__(256) quant_v_kernel(const uint16_t* __restrict
   constexpr int COPIES = kVTokens * SEG / 256;        // pieces copied per thread
   constexpr int RUNS = (D / 2) * (kVTokens / 16) / 256;  // (channel pair, 16-token run)s per thread
   __shared__ __align__(16) uint4 tile[kVTokens * SEG];
+  // the last prepass kernel: the mainloop that follows may start its set-up
+  // (it waits for this grid to complete before it reads anything written here)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // heads in the reverse of the statistics pass's order (its last rows are
   // still in L2)
   const int h = H - 1 - (int)blockIdx.y, b = (int)gridDim.z - 1 - (int)blockIdx.z;

@@ -557,6 +557,9 @@ __global__ void __launch_bounds__(kSThreads, kSCtasPerSm) prepass_stream_kernel(
   const uint32_t ts0 = smem_u32(tile);
   const uint8_t* tb = reinterpret_cast<const uint8_t*>(tile);
   int* pend = nullptr;  // thread 0: the count its previous SK or SV item still owes
+  // the mainloop that follows may start its set-up (it waits for this grid
+  // to complete before it reads anything written here)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     s_next = take(a);
     km_u = -1;

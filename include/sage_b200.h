@@ -44,6 +44,13 @@
  *     block at the start of the workspace; read them with
  *     sage_read_device_status.
  *   - Outputs are fully overwritten, padding included.
+ *   - Launch order: the last prepass kernel of sage_quant_qkv, sage_quant_v
+ *     and sage_attn_fwd lets the next kernel of the stream start early if
+ *     that kernel was launched as a programmatic dependent (CUDA's
+ *     programmatic stream serialization).  The library's mainloop is: it
+ *     waits (griddepcontrol.wait) for the prepass grid to complete before it
+ *     reads any quantised tensor.  A caller's own kernel launched that way
+ *     after a prepass call must wait in the same way before it reads them.
  *
  * Quantised buffer layouts (all 16-byte aligned, written by the prepasses):
  *   Nq = ceil(N/128)*128, Nk = ceil(N/64)*64, G32 = ceil(N/32), T64 = Nk/64

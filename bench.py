@@ -356,7 +356,7 @@ def main():
            torch.float32]
     qt = {n: torch.empty(s, dtype=dt, device=dev) for (n, s), dt in zip(shp.items(), dts)}
     if args.prepass == "auto":  # sage_attn_fwd's choice
-        args.prepass = "qkv" if 3 * B * H * N * D * 2 < (128 << 20) else "separate"
+        args.prepass = "qkv" if sage.sage_attn_fwd_prepass_kernels(B, N, H, D) == 1 else "separate"
     if args.prepass == "qkv":
         ws_pre = [sage.workspace(sage.SAGE_OP_QUANT_QKV, B, N, H, D, dev)]
         pre_kernels = sage.sage_quant_qkv_kernels(B, N, H, D)

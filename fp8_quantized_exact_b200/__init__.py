@@ -41,6 +41,7 @@ SAGE_STATUS_BYTES = 256
 
 # every symbol the header declares (the CPU test checks the exports)
 EXPORTS = ("sage_workspace_bytes", "sage_quant_qk", "sage_quant_v", "sage_quant_qkv", "sage_quant_qkv_kernels",
+           "sage_attn_fwd_prepass_kernels",
            "sage_norm_rope_quant_qk",
            "sage_attn_from_quant",
            "sage_attn_fwd", "sage_fwd_workspace_layout", "sage_read_device_status",
@@ -85,6 +86,7 @@ def lib():
             "sage_quant_v": [V, I, I, I, I, P, P, P, SZ, P],
             "sage_quant_qkv": [V, V, V, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P],
             "sage_quant_qkv_kernels": [I, I, I, I],
+            "sage_attn_fwd_prepass_kernels": [I, I, I, I],
             "sage_norm_rope_quant_qk": [V, V, P, P, P, P, ctypes.c_float, I, I, I, I, P, P, P, P, P, P, SZ, P],
             "sage_attn_from_quant": [P, P, P, P, P, P, P, L64, L64, L64, I, I, I, I,
                                      ctypes.c_float, P, SZ, P],
@@ -170,6 +172,15 @@ def sage_quant_qkv(q, k, v, q_i8, q_scale, k_i8, k_scale, k_mean, v_fp8, v_scale
                                 _ptr(workspace), workspace.numel() * workspace.element_size(),
                                 _stream(stream)),
            "sage_quant_qkv")
+
+
+def sage_attn_fwd_prepass_kernels(B, N, H, D):
+    """Prepass kernel launches of sage_attn_fwd for this shape (1: the single
+    launch, 6: the separate kernels; 0 for an empty shape)."""
+    n = lib().sage_attn_fwd_prepass_kernels(B, N, H, D)
+    if n < 0:
+        _check(n, "sage_attn_fwd_prepass_kernels")
+    return n
 
 
 def sage_quant_qkv_kernels(B, N, H, D):

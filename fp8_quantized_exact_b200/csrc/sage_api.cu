@@ -405,6 +405,13 @@ int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v, int B, 
                      workspace, kPrepStream, s);
 }
 
+int sage_attn_fwd_prepass_kernels(int B, int N, int H, int D) {
+  const int rc = check_dims(B, N, H, D);
+  if (rc) return rc;
+  if (empty(B, N, H)) return 0;
+  return prepass_impl(default_prepass(B, N, H, D)) == kPrepStream ? 1 : 6;
+}
+
 int sage_quant_qkv_kernels(int B, int N, int H, int D) {
   const int rc = check_dims(B, N, H, D);
   if (rc) return rc;

@@ -200,6 +200,15 @@ SAGE_API int sage_quant_qkv(sage_view_bf16 q, sage_view_bf16 k, sage_view_bf16 v
  * counterpart in the pages (launch accounting). */
 SAGE_API int sage_quant_qkv_kernels(int B, int N, int H, int D);
 
+/* Prepass kernel launches that sage_attn_fwd makes for this shape: 1 (the
+ * single launch of sage_quant_qkv, below about 128 MiB of Q, K and V) or 6
+ * (the separate kernels of sage_quant_qk and sage_quant_v); 0 for an empty
+ * shape; a negative SAGE_ERR_* for a shape the library refuses.  The
+ * SAGE_PREPASS environment variable ("separate" or "stream", read once)
+ * overrides the choice for every call.  No counterpart in the pages (launch
+ * accounting). */
+SAGE_API int sage_attn_fwd_prepass_kernels(int B, int N, int H, int D);
+
 /* Fused mainloop on quantised inputs: every 64-key tile in increasing order,
  * INT8 QK^T, score scaling, online softmax, E4M3 P, two K32 FP16 PV buffers
  * added into FP32, then 1/d, V scale and the BF16 store to `out`

@@ -288,3 +288,16 @@ def test_c_example_compiles(lib, tmp_path):
                          "-L/usr/local/cuda/lib64", "-lcudart", "-Wl,--no-undefined"],
                         capture_output=True, text=True)
     assert ld.returncode == 0, ld.stderr
+
+
+def test_attn_fwd_prepass_choice(lib):
+    """sage_attn_fwd's prepass: the single launch below 128 MiB of Q, K and V
+    (3*B*H*N*D BF16 values), the six separate kernels from there on."""
+    if os.environ.get("SAGE_PREPASS"):
+        pytest.skip("SAGE_PREPASS overrides the choice")
+    k = sage.sage_attn_fwd_prepass_kernels
+    assert k(1, 256, 2, 128) == 1 and k(1, 1000, 8, 128) == 1
+    assert k(2, 8192, 32, 128) == 6 and k(1, 37810, 56, 128) == 6 and k(4, 16384, 24, 64) == 6
+    assert k(1, 174762, 1, 128) == 1 and k(1, 174763, 1, 128) == 6  # 768 N bytes against 2^27
+    assert k(0, 10, 2, 64) == 0
+    assert lib.sage_attn_fwd_prepass_kernels(1, 10, 2, 96) == sage.SAGE_ERR_UNSUPPORTED
